@@ -1,0 +1,117 @@
+"""CPU oracle for prefill KV-cache token eviction (S1 * S2 scores, top-B select, gather).
+
+TEST INFRASTRUCTURE ONLY: the test-suite, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` are the only users. The product path (the package
+``token_eviction_b200``) never imports this module, and this module imports nothing
+from it; the two share only the seeded input generator ``synth``.
+
+The arithmetic lives in ``kvp_oracle.c``: the plain definition of the method in double
+precision, following "Preserving Large Activations: The Key to KV Cache Pruning"
+(SlimKV) Eq. 3 (S1), Eq. 4 (S2), Eq. 5 (S = S1 * S2) and Listing 1 (window_size,
+max_capacity_prompt), with C = sqrt(d) read from the CurDKV rebuttal page's statement
+of attention, softmax(Q K^T / C) V. This wrapper only marshals numpy arrays.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against closed forms,
+invariants, library routines and brute force.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvp_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile ``kvp_oracle.c`` into ``liboracle.so`` (gcc -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _get():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i, p = ctypes.c_int, ctypes.c_void_p
+        lib.oracle_score.argtypes = [i, i, i, i, i, i, p, p, p, p, p, p, p]
+        lib.oracle_score.restype = i
+        lib.oracle_select.argtypes = [i, i, i, i, p, p]
+        lib.oracle_select.restype = i
+        lib.oracle_compact.argtypes = [i, i, i, i, p, p, p, p, p]
+        lib.oracle_compact.restype = i
+        _lib = lib
+    return _lib
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, "bf16 tensors are passed as uint16 bit patterns"
+    return a
+
+
+def oracle_score(q_win, k, v, want_lse: bool = False):
+    """S1, S2, S [b, hkv, L] (float64) and optionally lse [b, hq, w].
+
+    q_win [b, hq, w, d], k and v [b, hkv, L, d]: bf16 bit patterns (uint16).
+    """
+    q_win, k, v = _u16(q_win), _u16(k), _u16(v)
+    b, hq, w, d = q_win.shape
+    _, hkv, L, _ = k.shape
+    assert k.shape == v.shape == (b, hkv, L, d)
+    s1 = np.empty((b, hkv, L))
+    s2 = np.empty((b, hkv, L))
+    s = np.empty((b, hkv, L))
+    lse = np.empty((b, hq, w)) if want_lse else None
+    rc = _get().oracle_score(b, hq, hkv, d, L, w, q_win.ctypes.data, k.ctypes.data, v.ctypes.data,
+                             s1.ctypes.data, s2.ctypes.data, s.ctypes.data,
+                             None if lse is None else lse.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_score: bad shape")
+    return (s1, s2, s, lse) if want_lse else (s1, s2, s)
+
+
+def oracle_select(score, window: int, budget: int):
+    """Kept positions [..., B] (int32, ascending) for scores [..., L] (any float dtype)."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    lead, L = score.shape[:-1], score.shape[-1]
+    rows = int(np.prod(lead)) if lead else 1
+    idx = np.empty(lead + (budget,), dtype=np.int32)
+    rc = _get().oracle_select(rows, L, window, budget, score.ctypes.data, idx.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_select: bad window/budget")
+    return idx
+
+
+def oracle_compact(k, v, idx):
+    """k_out, v_out [..., B, d] gathered row by row (bit copies)."""
+    k, v = _u16(k), _u16(v)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    L, d = k.shape[-2], k.shape[-1]
+    B = idx.shape[-1]
+    rows = int(np.prod(k.shape[:-2]))
+    k_out = np.empty(k.shape[:-2] + (B, d), dtype=np.uint16)
+    v_out = np.empty_like(k_out)
+    rc = _get().oracle_compact(rows, L, d, B, k.ctypes.data, v.ctypes.data, idx.ctypes.data,
+                               k_out.ctypes.data, v_out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_compact: index out of range")
+    return k_out, v_out
+
+
+def oracle_layer(q_win, k, v, window: int, budget: int):
+    """The whole path for one layer: scores, kept positions, compacted K and V."""
+    s1, s2, s = oracle_score(q_win, k, v)
+    idx = oracle_select(s, window, budget)
+    k_out, v_out = oracle_compact(k, v, idx)
+    return {"s1": s1, "s2": s2, "score": s, "idx": idx, "k_out": k_out, "v_out": v_out}

@@ -1,0 +1,174 @@
+/*
+ * CPU oracle for prefill KV-cache token eviction by S1 * S2 scores.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load this
+ * file: only the test-suite, the smoke check and the benchmark's CPU-baseline leg use
+ * it. It shares no code with the CUDA library.
+ *
+ * It is the plain definition, written for a reader to check by eye, in double
+ * precision, one (sequence, KV head) at a time (OpenMP over those independent units):
+ *
+ *   "Preserving Large Activations: The Key to KV Cache Pruning" (SlimKV), Section 3:
+ *     Eq. 3  S1[j] = sum over the query heads g of the KV head's GQA group (Section 3.1,
+ *                    "grouped-wise" scoring) and over the queries i of the observation
+ *                    window of softmax_j(q_{g,i} . k_j / C)
+ *     Eq. 4  S2[j] = max over the head dimension of |V[j, :]|
+ *     Eq. 5  S[j]  = S1[j] * S2[j]
+ *     Listing 1: hyperparameters window_size (w) and max_capacity_prompt (B).
+ *   CurDKV rebuttal page (paperhub.cn/paper/klmc4fwPLd), "Clarification of the claims in
+ *   Section 3.1": attention is softmax(Q K^T / C) V with C a constant of the dimension;
+ *   read here as C = sqrt(d).
+ *
+ * Readings taken where the pages are silent:
+ *   - window query i (0 <= i < w) sits at absolute position p_i = L - w + i and sees keys
+ *     j <= p_i (causal prefill);
+ *   - B counts every kept position, the w window positions included; the other B - w
+ *     are the highest-S positions among j < L - w, ties going to the lower j;
+ *   - kept positions are listed in ascending order;
+ *   - query head hq belongs to KV head hq / G, G = Hq / Hkv.
+ *
+ * bf16 inputs arrive as their 16-bit patterns and are widened exactly to double.
+ *
+ * Parity pins (tests): sum_j S1 = G w; closed forms for identical keys and for a
+ * single planted key; G = 1, w = 1 against a library softmax; brute force on tiny
+ * inputs; selection against a library stable sort; gather against library indexing.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double widen_bf16(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/*
+ * Scores of every position j in [0, L) of every (sequence b, KV head h).
+ *   q      [batch, hq, w, d]   bf16 bits, the last w queries of the prefill
+ *   k, v   [batch, hkv, L, d]  bf16 bits
+ *   s1, s2, score [batch, hkv, L]  double (s1, s2 may be NULL)
+ *   lse    [batch, hq, w] double, log-sum-exp of each window query's logits (may be NULL)
+ * Returns 0, or -1 on a bad shape.
+ */
+int oracle_score(int batch, int hq, int hkv, int d, int L, int w,
+                 const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                 double* s1_out, double* s2_out, double* score, double* lse_out) {
+    if (batch < 1 || hkv < 1 || hq % hkv || d < 1 || w < 1 || w > L) return -1;
+    const int G = hq / hkv;
+    const double C = sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < batch * hkv; ++bh) {
+        const int b = bh / hkv, h = bh % hkv;
+        const uint16_t* kh = k + (size_t)bh * L * d;
+        const uint16_t* vh = v + (size_t)bh * L * d;
+        double* s1 = (double*)calloc((size_t)L, sizeof(double));
+        double* logit = (double*)malloc((size_t)L * sizeof(double));
+        double* qrow = (double*)malloc((size_t)d * sizeof(double));
+        double* kd = (double*)malloc((size_t)L * d * sizeof(double));
+        for (size_t e = 0; e < (size_t)L * d; ++e) kd[e] = widen_bf16(kh[e]);
+
+        /* Eq. 3: one softmax row per (query head g of the group, window query i). */
+        for (int g = 0; g < G; ++g) {
+            const int head_q = h * G + g;
+            for (int i = 0; i < w; ++i) {
+                const uint16_t* qi = q + (((size_t)b * hq + head_q) * w + i) * d;
+                for (int c = 0; c < d; ++c) qrow[c] = widen_bf16(qi[c]);
+                const int p = L - w + i; /* causal: keys 0..p are visible */
+                double mx = -INFINITY;
+                for (int j = 0; j <= p; ++j) {
+                    double dot = 0.0;
+                    for (int c = 0; c < d; ++c) dot += qrow[c] * kd[(size_t)j * d + c];
+                    logit[j] = dot / C;
+                    if (logit[j] > mx) mx = logit[j];
+                }
+                double sum = 0.0;
+                for (int j = 0; j <= p; ++j) sum += exp(logit[j] - mx);
+                const double lse = mx + log(sum);
+                if (lse_out) lse_out[((size_t)b * hq + head_q) * w + i] = lse;
+                for (int j = 0; j <= p; ++j) s1[j] += exp(logit[j] - lse);
+            }
+        }
+        /* Eq. 4 and Eq. 5. */
+        for (int j = 0; j < L; ++j) {
+            double m = 0.0;
+            for (int c = 0; c < d; ++c) {
+                double a = fabs(widen_bf16(vh[(size_t)j * d + c]));
+                if (a > m) m = a;
+            }
+            const size_t o = (size_t)bh * L + j;
+            if (s1_out) s1_out[o] = s1[j];
+            if (s2_out) s2_out[o] = m;
+            score[o] = s1[j] * m;
+        }
+        free(kd);
+        free(qrow);
+        free(logit);
+        free(s1);
+    }
+    return 0;
+}
+
+typedef struct {
+    double s;
+    int32_t j;
+} cand_t;
+
+/* Higher score first; equal scores: lower position first. */
+static int by_score_then_pos(const void* a, const void* b) {
+    const cand_t* x = (const cand_t*)a;
+    const cand_t* y = (const cand_t*)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+/*
+ * Kept positions of every (b, h) row: the w window positions [L-w, L) and the B - w
+ * highest-scoring positions of [0, L-w), listed in ascending order.
+ *   score [rows, L] double;  idx [rows, B] int32.
+ * Returns 0, or -1 on a bad shape.
+ */
+int oracle_select(int rows, int L, int w, int B, const double* score, int32_t* idx) {
+    if (rows < 0 || w < 1 || w > L || B < w || B > L) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < rows; ++r) {
+        const double* s = score + (size_t)r * L;
+        const int n = L - w, kk = B - w;
+        cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)(n > 0 ? n : 1));
+        unsigned char* keep = (unsigned char*)calloc((size_t)L, 1);
+        for (int j = 0; j < n; ++j) {
+            c[j].s = s[j];
+            c[j].j = j;
+        }
+        qsort(c, (size_t)n, sizeof(cand_t), by_score_then_pos);
+        for (int t = 0; t < kk; ++t) keep[c[t].j] = 1;
+        for (int j = n; j < L; ++j) keep[j] = 1;
+        int32_t* out = idx + (size_t)r * B;
+        int t = 0;
+        for (int j = 0; j < L; ++j)
+            if (keep[j]) out[t++] = j;
+        free(keep);
+        free(c);
+    }
+    return 0;
+}
+
+/*
+ * Compaction: k_out[r, t, :] = k[r, idx[r, t], :] and the same for v, as a copy of the
+ * 16-bit patterns.  k, v [rows, L, d];  idx [rows, B];  k_out, v_out [rows, B, d].
+ * Returns 0, or -1 if an index lies outside [0, L).
+ */
+int oracle_compact(int rows, int L, int d, int B, const uint16_t* k, const uint16_t* v,
+                   const int32_t* idx, uint16_t* k_out, uint16_t* v_out) {
+    for (int r = 0; r < rows; ++r)
+        for (int t = 0; t < B; ++t) {
+            const int32_t j = idx[(size_t)r * B + t];
+            if (j < 0 || j >= L) return -1;
+            memcpy(k_out + ((size_t)r * B + t) * d, k + ((size_t)r * L + j) * d, sizeof(uint16_t) * d);
+            memcpy(v_out + ((size_t)r * B + t) * d, v + ((size_t)r * L + j) * d, sizeof(uint16_t) * d);
+        }
+    return 0;
+}

@@ -1,0 +1,242 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each test fixes a result by mathematics or by a library routine, so that a plausible
+slip in the oracle (a dropped term, a wrong scale, a wrong causal index, a wrong GQA
+head mapping, a transposed operand, a wrong tie rule) fails at least one of them:
+
+* the softmax rows of Eq. 3 each sum to 1, so sum_j S1[j] = G w;
+* identical keys make every visible logit equal, giving S1 in closed form (harmonic
+  sums that depend on the causal mask inside the window);
+* a single planted key along one axis gives each softmax row in closed form, with
+  per-query-head amplitudes that expose the GQA mapping and the scale C = sqrt(d);
+* G = 1, w = 1 reduces Eq. 3 to one softmax row, compared with torch.softmax (fp64)
+  and the log-sum-exp with scipy;
+* planted |V| values give Eq. 4 exactly;
+* selection against numpy's stable lexsort, compaction against numpy indexing;
+* brute force with math.fsum on tiny inputs.
+
+All run on the CPU (no GPU mark).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+
+def bf16(x):
+    return synth.round_bf16(np.asarray(x, dtype=np.float64))
+
+
+def f64(bits):
+    return synth.bf16_to_f64(bits)
+
+
+def rand_inputs(b, hq, hkv, d, L, w, seed=7):
+    rng = np.random.default_rng(seed)
+    q = bf16(rng.standard_normal((b, hq, w, d)))
+    k = bf16(rng.standard_normal((b, hkv, L, d)))
+    v = bf16(rng.standard_normal((b, hkv, L, d)))
+    return q, k, v
+
+
+@pytest.mark.parametrize("b,hq,hkv,d,L,w", [(1, 4, 2, 64, 96, 8), (2, 6, 2, 32, 50, 7), (1, 2, 2, 16, 9, 9)])
+def test_s1_total_is_g_times_w(b, hq, hkv, d, L, w):
+    q, k, v = rand_inputs(b, hq, hkv, d, L, w)
+    s1, s2, s = oracle.oracle_score(q, k, v)
+    G = hq // hkv
+    np.testing.assert_allclose(s1.sum(-1), G * w, rtol=1e-12)
+    assert (s1 >= 0).all()
+
+
+def test_identical_keys_closed_form():
+    b, hq, hkv, d, L, w = 1, 6, 2, 64, 40, 6
+    G = hq // hkv
+    rng = np.random.default_rng(3)
+    q = bf16(rng.standard_normal((b, hq, w, d)))
+    row = bf16(rng.standard_normal(d))
+    k = np.broadcast_to(row, (b, hkv, L, d)).copy()
+    v = bf16(rng.standard_normal((b, hkv, L, d)))
+    s1, _, _ = oracle.oracle_score(q, k, v)
+    pos = [L - w + i for i in range(w)]
+    expect = np.empty(L)
+    for j in range(L):
+        # row i sees p_i + 1 equal logits, so each visible key gets 1 / (p_i + 1)
+        expect[j] = G * sum(1.0 / (p + 1) for p in pos if j <= p)
+    for h in range(hkv):
+        np.testing.assert_allclose(s1[0, h], expect, rtol=1e-12)
+
+
+def test_planted_key_closed_form_gqa_mapping_and_scale():
+    b, hq, hkv, d, L, w = 1, 6, 3, 64, 30, 4
+    G = hq // hkv
+    amp = [2.0, 4.0, 8.0, 16.0, 3.0, 6.0]   # one amplitude per query head, exact in bf16
+    planted = [5, 11, 27]                   # the key position planted in each KV head
+    q = np.zeros((b, hq, w, d))
+    for hqi in range(hq):
+        q[0, hqi, :, 0] = amp[hqi]
+    k = np.zeros((b, hkv, L, d))
+    for h in range(hkv):
+        k[0, h, planted[h], 0] = 1.0
+    v = np.ones((b, hkv, L, d))
+    s1, s2, s = oracle.oracle_score(bf16(q), bf16(k), bf16(v))
+    C = math.sqrt(d)
+    for h in range(hkv):
+        jstar = planted[h]
+        expect = np.zeros(L)
+        for g in range(G):
+            x = amp[h * G + g] / C          # query head h*G+g belongs to KV head h
+            for i in range(w):
+                p = L - w + i
+                if jstar <= p:
+                    den = math.exp(x) + p   # one key at logit x, p keys at logit 0
+                    for j in range(p + 1):
+                        expect[j] += (math.exp(x) if j == jstar else 1.0) / den
+                else:
+                    for j in range(p + 1):
+                        expect[j] += 1.0 / (p + 1)
+        np.testing.assert_allclose(s1[0, h], expect, rtol=1e-12)
+        np.testing.assert_array_equal(s2[0, h], 1.0)
+        np.testing.assert_allclose(s[0, h], expect, rtol=1e-12)
+
+
+def test_single_query_reduces_to_library_softmax():
+    import torch
+    from scipy.special import logsumexp
+    b, hq, hkv, d, L, w = 2, 3, 3, 128, 257, 1
+    q, k, v = rand_inputs(b, hq, hkv, d, L, w, seed=11)
+    s1, s2, s, lse = oracle.oracle_score(q, k, v, want_lse=True)
+    qf, kf = f64(q), f64(k)
+    for bi in range(b):
+        for h in range(hkv):
+            logits = torch.from_numpy(kf[bi, h] @ qf[bi, h, 0]) / math.sqrt(d)
+            ref = torch.softmax(logits, dim=0).numpy()
+            np.testing.assert_allclose(s1[bi, h], ref, rtol=1e-12, atol=1e-300)
+            np.testing.assert_allclose(lse[bi, h, 0], logsumexp(logits.numpy()), rtol=1e-13)
+
+
+def test_s2_planted_abs_max():
+    b, hkv, L, d = 1, 2, 20, 16
+    rng = np.random.default_rng(5)
+    v = rng.uniform(-0.5, 0.5, (b, hkv, L, d))
+    expect = np.empty((b, hkv, L))
+    for h in range(hkv):
+        for j in range(L):
+            val = (j + 1) * (0.25 if h == 0 else 0.75)
+            sign = -1.0 if (j + h) % 2 else 1.0       # negative planted values: |.| matters
+            v[0, h, j, (3 * j + h) % d] = sign * val
+            expect[0, h, j] = max(val, 0.5) if val < 0.5 else val
+    vb = bf16(v)
+    # bf16 rounding of the planted values is exact (multiples of 1/4 below 256)
+    q = bf16(rng.standard_normal((b, 2 * hkv, 2, d)))
+    k = bf16(rng.standard_normal((b, hkv, L, d)))
+    _, s2, _ = oracle.oracle_score(q, k, vb)
+    ref = np.abs(f64(vb)).max(-1)                 # library max as a second witness
+    np.testing.assert_array_equal(s2, ref)
+    big = expect >= 0.5
+    np.testing.assert_array_equal(s2[big], expect[big])
+
+
+def brute_force(q, k, v):
+    b, hq, w, d = q.shape
+    _, hkv, L, _ = k.shape
+    G = hq // hkv
+    qf, kf, vf = f64(q), f64(k), f64(v)
+    s1 = np.zeros((b, hkv, L))
+    for bi in range(b):
+        for h in range(hkv):
+            for g in range(G):
+                for i in range(w):
+                    p = L - w + i
+                    lg = [math.fsum(qf[bi, h * G + g, i, c] * kf[bi, h, j, c] for c in range(d)) / math.sqrt(d)
+                          for j in range(p + 1)]
+                    m = max(lg)
+                    den = math.fsum(math.exp(x - m) for x in lg)
+                    for j in range(p + 1):
+                        s1[bi, h, j] += math.exp(lg[j] - m) / den
+    s2 = np.abs(vf).max(-1)
+    return s1, s2, s1 * s2
+
+
+def test_brute_force_tiny():
+    q, k, v = rand_inputs(2, 4, 2, 8, 24, 5, seed=21)
+    s1, s2, s = oracle.oracle_score(q, k, v)
+    r1, r2, r = brute_force(q, k, v)
+    np.testing.assert_allclose(s1, r1, rtol=1e-12)
+    np.testing.assert_array_equal(s2, r2)
+    np.testing.assert_allclose(s, r, rtol=1e-12)
+
+
+def library_select(score, w, B):
+    L = score.shape[-1]
+    out = []
+    for row in score.reshape(-1, L):
+        n = L - w
+        order = np.lexsort((np.arange(n), -row[:n]))   # by -score, then by position
+        keep = np.sort(np.concatenate([order[:B - w], np.arange(n, L)]))
+        out.append(keep)
+    return np.array(out, dtype=np.int32).reshape(score.shape[:-1] + (B,))
+
+
+@pytest.mark.parametrize("L,w,B", [(100, 8, 30), (64, 1, 1), (64, 4, 64), (50, 50, 50), (33, 5, 5)])
+def test_select_matches_library_sort(L, w, B):
+    rng = np.random.default_rng(L + w + B)
+    score = rng.random((3, 2, L))
+    score[0, 0, 10:20] = 0.5                      # a block of exact ties
+    idx = oracle.oracle_select(score, w, B)
+    np.testing.assert_array_equal(idx, library_select(score, w, B))
+    assert idx.shape == (3, 2, B)
+    assert (np.diff(idx, axis=-1) > 0).all()      # strictly ascending
+    assert (idx[..., B - w:] == np.arange(L - w, L)).all()
+
+
+def test_select_ties_go_to_lower_position():
+    L, w, B = 40, 4, 14
+    score = np.full((1, L), 2.0)
+    idx = oracle.oracle_select(score, w, B)
+    np.testing.assert_array_equal(idx[0], np.r_[np.arange(B - w), np.arange(L - w, L)])
+
+
+def test_compact_matches_library_indexing():
+    rng = np.random.default_rng(9)
+    k = rng.integers(0, 65536, (2, 3, 50, 16), dtype=np.uint16)
+    v = rng.integers(0, 65536, (2, 3, 50, 16), dtype=np.uint16)
+    idx = np.sort(rng.permuted(np.tile(np.arange(50), (6, 1)), axis=1)[:, :12], axis=1).reshape(2, 3, 12).astype(np.int32)
+    ko, vo = oracle.oracle_compact(k, v, idx)
+    np.testing.assert_array_equal(ko, np.take_along_axis(k, idx[..., None].astype(np.int64), axis=2))
+    np.testing.assert_array_equal(vo, np.take_along_axis(v, idx[..., None].astype(np.int64), axis=2))
+
+
+def test_planted_needle_and_value_outlier_are_kept():
+    b, hq, hkv, d, L, w, B = 1, 4, 2, 64, 300, 8, 20
+    q, k, v = rand_inputs(b, hq, hkv, d, L, w, seed=13)
+    qf = f64(q)
+    needle, outlier = 37, 201
+    for h in range(hkv):
+        qq = qf[0, h * 2 + 1, 3]
+        k[0, h, needle] = bf16(24 * math.sqrt(d) * qq / (qq @ qq))   # logit 24 for that query
+        v[0, h, outlier] = bf16(f64(v[0, h, outlier]) * 1000)
+    out = oracle.oracle_layer(q, k, v, w, B)
+    for h in range(hkv):
+        assert needle in out["idx"][0, h]
+        assert outlier in out["idx"][0, h]
+    assert out["idx"].shape == (1, 2, B)
+
+
+def test_identity_when_budget_is_context():
+    q, k, v = rand_inputs(1, 2, 1, 16, 33, 3)
+    out = oracle.oracle_layer(q, k, v, 3, 33)
+    np.testing.assert_array_equal(out["idx"][0, 0], np.arange(33))
+    np.testing.assert_array_equal(out["k_out"], k)
+
+
+def test_bad_shapes_raise():
+    q, k, v = rand_inputs(1, 2, 1, 16, 10, 3)
+    with pytest.raises(ValueError):
+        oracle.oracle_select(np.zeros((1, 10)), 3, 2)      # B < w
+    with pytest.raises(ValueError):
+        oracle.oracle_select(np.zeros((1, 10)), 3, 11)     # B > L
+    with pytest.raises(ValueError):
+        oracle.oracle_compact(k, v, np.array([[[0, 10]]], dtype=np.int32))
