@@ -1,0 +1,117 @@
+/*
+ * kvp.h - prefill KV-cache token eviction on NVIDIA B200 (sm_100a): C ABI.
+ *
+ * The method ("Preserving Large Activations: The Key to KV Cache Pruning", SlimKV,
+ * Section 3) scores every cached position j of every KV head with S = S1 * S2:
+ *
+ *   S1[j]  (Eq. 3) the softmax attention weight that each of the last w queries of the
+ *          prefill (the observation window) gives key j, summed over those queries and
+ *          over the G query heads that share the KV head (Section 3.1, grouped-wise
+ *          scoring for GQA). The softmax is the attention softmax(q . k / C) with
+ *          C = sqrt(d) (the CurDKV rebuttal page's statement of attention). Window query
+ *          i sits at position L - w + i and sees keys j <= L - w + i.
+ *   S2[j]  (Eq. 4) the largest |V[j, c]| over the head dimension c, so positions that
+ *          carry large activations in the value cache survive.
+ *   S[j]   (Eq. 5) S1[j] * S2[j].
+ *
+ * It then keeps B positions per (sequence, KV head) - Listing 1's window_size (w) and
+ * max_capacity_prompt (B): the w window positions always, plus the B - w highest-S
+ * positions before the window - and compacts K and V to those rows.
+ *
+ * Conventions for every call:
+ *   - All tensors are device memory, contiguous, row-major, innermost dimension last.
+ *     bf16 tensors are passed as their 16-bit patterns (uint16_t).
+ *   - Query head hq belongs to KV head hq / G, G = hq_count / hkv_count.
+ *   - The caller owns and allocates every buffer. The library allocates no device
+ *     memory and keeps no state between calls; calls with distinct workspaces may run
+ *     concurrently from several host threads.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls only enqueue
+ *     work and never synchronise the host.
+ *   - Argument errors are detected on the host before anything is launched; the outputs
+ *     are then untouched. A launch failure returns KVP_ERR_CUDA (the CUDA error is
+ *     consumed). Kernels contain no waits that can hang.
+ */
+#ifndef KVP_H_
+#define KVP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVP_API __attribute__((visibility("default")))
+#else
+#define KVP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem shape. budget (B) counts every kept position, window included. */
+typedef struct {
+    int32_t batch;     /* b   >= 1 */
+    int32_t hq;        /* query heads, a multiple of hkv */
+    int32_t hkv;       /* KV heads >= 1 */
+    int32_t head_dim;  /* d: 64 or 128 */
+    int32_t seq_len;   /* L >= 1 */
+    int32_t window;    /* w: 1 <= w <= L, and G * w <= 512 */
+    int32_t budget;    /* B: w <= B <= L */
+} kvp_shape;
+
+typedef enum {
+    KVP_OK = 0,
+    KVP_ERR_NULL = 1,      /* a required pointer is NULL */
+    KVP_ERR_SHAPE = 2,     /* shape outside the limits above */
+    KVP_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned */
+    KVP_ERR_WORKSPACE = 4, /* workspace NULL or smaller than kvp_workspace_bytes() */
+    KVP_ERR_CUDA = 5,      /* a CUDA runtime/driver call or kernel launch failed */
+    KVP_ERR_TIMEOUT = 6    /* reserved: a bounded device-side wait gave up */
+} kvp_status;
+
+/* Bytes of device workspace that kvp_score and kvp_select need for `shape`
+ * (split-L softmax partials, log-sum-exp values, selection scratch); 0 for an invalid
+ * shape. The workspace holds no state between calls. */
+KVP_API size_t kvp_workspace_bytes(const kvp_shape* shape);
+
+/*
+ * Scores S, and optionally S1 and S2, of every position (window included).
+ *   q_win  [b, hq, w, d]   bf16: the last w queries of the prefill, Q[:, :, L-w:, :]
+ *   k, v   [b, hkv, L, d]  bf16: the layer's key and value cache
+ *   score  [b, hkv, L]     fp32 output, S = S1 * S2
+ *   s1, s2 [b, hkv, L]     fp32 outputs, may be NULL
+ *   workspace  device scratch of at least kvp_workspace_bytes(shape) bytes
+ * Arithmetic: bf16 products accumulated in fp32, fp32 exponentials.
+ */
+KVP_API kvp_status kvp_score(const kvp_shape* shape, const uint16_t* q_win, const uint16_t* k,
+                             const uint16_t* v, float* score, float* s1, float* s2,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Kept positions of every (b, KV head): the B - w highest scores among positions
+ * [0, L - w) (equal scores: lower position first) and the window [L - w, L), listed in
+ * ascending position order.
+ *   score [b, hkv, L] fp32, non-negative (as kvp_score writes it)
+ *   idx   [b, hkv, B] int32 output
+ * B == L gives the identity; B == w keeps the window alone.
+ */
+KVP_API kvp_status kvp_select(const kvp_shape* shape, const float* score, int32_t* idx,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Compaction: k_out[b, h, t, :] = k[b, h, idx[b, h, t], :], the same for v; a bit copy.
+ *   k, v          [b, hkv, L, d] bf16
+ *   idx           [b, hkv, B]    int32, entries in [0, L) (an entry outside that range
+ *                                yields a zero row instead of an out-of-bounds read)
+ *   k_out, v_out  [b, hkv, B, d] bf16 outputs; must not overlap k or v
+ */
+KVP_API kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
+                               const int32_t* idx, uint16_t* k_out, uint16_t* v_out, void* stream);
+
+/* A static, human-readable name of a status code. */
+KVP_API const char* kvp_status_string(kvp_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVP_H_ */

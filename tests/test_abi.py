@@ -1,0 +1,91 @@
+"""The C-ABI library loads, exports what include/kvp.h declares, and rejects bad
+arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"KVP_API\s+[\w\s\*]*?\b(kvp_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_boundary():
+    assert {"kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact",
+            "kvp_status_string"} <= declared_symbols()
+
+
+def test_library_exports_every_declared_symbol():
+    import token_eviction_b200 as m
+    lib = ctypes.CDLL(m.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} declared but not exported"
+
+
+def test_status_strings():
+    import token_eviction_b200 as m
+    for code, name in m.STATUS_NAMES.items():
+        assert m.kvp_status_string(code).startswith(name)
+    assert "unknown" in m.kvp_status_string(99)
+
+
+def test_workspace_bytes_positive_and_zero_for_bad_shapes():
+    import token_eviction_b200 as m
+    assert m.kvp_workspace_bytes((1, 32, 8, 128, 32768, 32, 2048)) > 0
+    assert m.kvp_workspace_bytes((8, 28, 4, 128, 16384, 64, 1024)) > 0
+    bad = [(1, 32, 7, 128, 1024, 32, 64),    # hq not a multiple of hkv
+           (1, 32, 8, 96, 1024, 32, 64),     # unsupported head_dim
+           (1, 32, 8, 128, 1024, 32, 16),    # B < w
+           (1, 32, 8, 128, 1024, 32, 1025),  # B > L
+           (1, 32, 8, 128, 16, 32, 32),      # w > L
+           (1, 32, 1, 128, 4096, 32, 64),    # G * w > 512
+           (0, 32, 8, 128, 1024, 32, 64)]
+    for s in bad:
+        assert m.kvp_workspace_bytes(s) == 0, s
+
+
+def raw(m):
+    return ctypes.CDLL(m.LIB_PATH)
+
+
+def call_score(m, shape, q=16, k=16, v=16, score=16, ws=16, ws_bytes=1 << 30):
+    lib = m._lib
+    sh = m.make_shape(*shape)
+    return lib.kvp_score(ctypes.byref(sh), q, k, v, score, None, None, ws, ws_bytes, None)
+
+
+def test_host_side_argument_errors():
+    import token_eviction_b200 as m
+    ok_shape = (1, 32, 8, 128, 4096, 32, 256)
+    assert call_score(m, ok_shape, q=None) == 1
+    assert call_score(m, ok_shape, score=None) == 1
+    assert m._lib.kvp_score(None, 16, 16, 16, 16, None, None, 16, 1 << 30, None) == 1
+    assert call_score(m, (1, 32, 8, 100, 4096, 32, 256)) == 2
+    assert call_score(m, ok_shape, k=24) == 3          # misaligned
+    assert call_score(m, ok_shape, ws=None) == 4
+    assert call_score(m, ok_shape, ws_bytes=8) == 4
+    sh = m.make_shape(*ok_shape)
+    assert m._lib.kvp_select(ctypes.byref(sh), 16, None, 16, 1 << 30, None) == 1
+    assert m._lib.kvp_select(ctypes.byref(sh), 16, 20, 16, 1 << 30, None) == 3
+    assert m._lib.kvp_select(ctypes.byref(sh), 16, 16, 16, 0, None) == 4
+    assert m._lib.kvp_compact(ctypes.byref(sh), 16, 16, 16, 16, None, None) == 1
+    assert m._lib.kvp_compact(ctypes.byref(sh), 16, 16, 16, 16, 8, None) == 3
+    bad = m.make_shape(1, 32, 8, 128, 4096, 32, 8)
+    assert m._lib.kvp_compact(ctypes.byref(bad), 16, 16, 16, 16, 16, None) == 2
+
+
+def test_binding_validates_tensors_before_calling():
+    import torch
+    import token_eviction_b200 as m
+    sh = m.make_shape(1, 4, 2, 64, 128, 16, 32)
+    cpu = torch.zeros((1, 4, 16, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        m.kvp_score(sh, cpu, cpu, cpu, cpu)

@@ -1,0 +1,128 @@
+// C ABI of the kvp library: argument checks, workspace layout, launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "kvp.h"
+#include "kvp_internal.cuh"
+
+namespace kvp {
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+        return n;
+    return 148;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static bool shape_ok(const kvp_shape& s) {
+    if (s.batch < 1 || s.hkv < 1 || s.hq < 1 || s.hq % s.hkv != 0) return false;
+    if (s.head_dim != 64 && s.head_dim != 128) return false;
+    if (s.seq_len < 1 || s.window < 1 || s.window > s.seq_len) return false;
+    if (s.budget < s.window || s.budget > s.seq_len) return false;
+    if ((int64_t)(s.hq / s.hkv) * s.window > kMaxGroupRows) return false;
+    // element offsets of k/v stay well inside int64; row counts inside int32
+    if ((int64_t)s.batch * s.hkv > 65535) return false;  // grid y extent
+    if ((int64_t)s.batch * s.hkv * s.seq_len > INT32_MAX) return false;
+    if ((int64_t)s.batch * s.hq * s.window > INT32_MAX) return false;
+    return true;
+}
+
+bool plan_of(const kvp_shape& s, Plan* p) {
+    if (!shape_ok(s)) return false;
+    p->G = s.hq / s.hkv;
+    p->rows = p->G * s.window;
+    // Split L so that the log-sum-exp pass has about two CTAs per SM; splits are whole
+    // multiples of 128 keys. The split count does not depend on the device.
+    const int64_t units = (int64_t)s.batch * s.hkv;
+    const int tiles = (s.seq_len + 127) / 128;
+    int64_t want = (2 * 148 + units - 1) / units;
+    int nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(want, tiles));
+    int tiles_per_split = (tiles + nsplit - 1) / nsplit;
+    nsplit = (tiles + tiles_per_split - 1) / tiles_per_split;
+    p->nsplit = nsplit;
+    p->keys_per_split = tiles_per_split * 128;
+    size_t off = 0;
+    p->off_part = off;
+    off += align_up((size_t)s.batch * s.hq * s.window * nsplit * sizeof(float2), 256);
+    p->off_select = off;
+    off += 256;
+    p->bytes = off;
+    return true;
+}
+
+}  // namespace kvp
+
+using namespace kvp;
+
+static bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+extern "C" size_t kvp_workspace_bytes(const kvp_shape* shape) {
+    Plan p;
+    if (!shape || !plan_of(*shape, &p)) return 0;
+    return p.bytes;
+}
+
+extern "C" kvp_status kvp_score(const kvp_shape* shape, const uint16_t* q_win, const uint16_t* k,
+                                const uint16_t* v, float* score, float* s1, float* s2,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    if (!shape || !q_win || !k || !v || !score) return KVP_ERR_NULL;
+    Plan p;
+    if (!plan_of(*shape, &p)) return KVP_ERR_SHAPE;
+    if (!aligned16(q_win) || !aligned16(k) || !aligned16(v) || !aligned16(score) ||
+        !aligned16(s1) || !aligned16(s2))
+        return KVP_ERR_ALIGN;
+    if (!workspace || workspace_bytes < p.bytes) return KVP_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KVP_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    float2* part = (float2*)((char*)workspace + p.off_part);
+    if (launch_lse_partial(*shape, p, q_win, k, part, st) != cudaSuccess) return KVP_ERR_CUDA;
+    if (launch_score(*shape, p, q_win, k, v, part, score, s1, s2, st) != cudaSuccess)
+        return KVP_ERR_CUDA;
+    return KVP_OK;
+}
+
+extern "C" kvp_status kvp_select(const kvp_shape* shape, const float* score, int32_t* idx,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    if (!shape || !score || !idx) return KVP_ERR_NULL;
+    Plan p;
+    if (!plan_of(*shape, &p)) return KVP_ERR_SHAPE;
+    if (!aligned16(score) || !aligned16(idx)) return KVP_ERR_ALIGN;
+    if (!workspace || workspace_bytes < p.bytes) return KVP_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KVP_ERR_ALIGN;
+    if (launch_select(*shape, p, score, idx, (char*)workspace + p.off_select,
+                      (cudaStream_t)stream) != cudaSuccess)
+        return KVP_ERR_CUDA;
+    return KVP_OK;
+}
+
+extern "C" kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
+                                  const int32_t* idx, uint16_t* k_out, uint16_t* v_out,
+                                  void* stream) {
+    if (!shape || !k || !v || !idx || !k_out || !v_out) return KVP_ERR_NULL;
+    Plan p;
+    if (!plan_of(*shape, &p)) return KVP_ERR_SHAPE;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(k_out) ||
+        !aligned16(v_out))
+        return KVP_ERR_ALIGN;
+    if (launch_compact(*shape, k, v, idx, k_out, v_out, (cudaStream_t)stream) != cudaSuccess)
+        return KVP_ERR_CUDA;
+    return KVP_OK;
+}
+
+extern "C" const char* kvp_status_string(kvp_status status) {
+    switch (status) {
+        case KVP_OK: return "KVP_OK";
+        case KVP_ERR_NULL: return "KVP_ERR_NULL: a required pointer is NULL";
+        case KVP_ERR_SHAPE: return "KVP_ERR_SHAPE: shape outside the supported limits";
+        case KVP_ERR_ALIGN: return "KVP_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case KVP_ERR_WORKSPACE: return "KVP_ERR_WORKSPACE: workspace missing or too small";
+        case KVP_ERR_CUDA: return "KVP_ERR_CUDA: a CUDA call or kernel launch failed";
+        case KVP_ERR_TIMEOUT: return "KVP_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "unknown kvp_status";
+}

@@ -1,0 +1,53 @@
+// Compaction of the K/V cache to the kept positions: a 16-byte vectorised row gather.
+//
+// k_out[b, h, t, :] = k[b, h, idx[b, h, t], :] and the same for v, as a bit copy (the
+// eviction step of "Preserving Large Activations: The Key to KV Cache Pruning",
+// Listing 1: the cache keeps max_capacity_prompt positions). Each thread moves one
+// 16-byte piece of one kept K row and the same piece of the V row; a grid of
+// whole waves over the SMs strides over all pieces.
+#include <cuda_runtime.h>
+
+#include "kvp_internal.cuh"
+
+namespace kvp {
+namespace {
+
+__global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ k,
+                                                   const uint4* __restrict__ v,
+                                                   const int32_t* __restrict__ idx,
+                                                   uint4* __restrict__ k_out,
+                                                   uint4* __restrict__ v_out, int L, int B,
+                                                   int vec_per_row, long long total) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+        const long long rt = e / vec_per_row;  // (row, t)
+        const int c = (int)(e - rt * vec_per_row);
+        const long long row = rt / B;
+        const int j = __ldg(idx + rt);
+        uint4 a = make_uint4(0, 0, 0, 0), b = a;
+        if (j >= 0 && j < L) {
+            const long long src = (row * L + j) * vec_per_row + c;
+            a = __ldg(k + src);
+            b = __ldg(v + src);
+        }
+        __stcs(k_out + e, a);
+        __stcs(v_out + e, b);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t* v,
+                           const int32_t* idx, uint16_t* k_out, uint16_t* v_out, cudaStream_t st) {
+    const int vec_per_row = s.head_dim * 2 / 16;
+    const long long total = (long long)s.batch * s.hkv * s.budget * vec_per_row;
+    const long long want = (total + 255) / 256;
+    const int sms = num_sms();
+    const long long cap = (long long)sms * 8;  // 8 resident CTAs of 256 threads per SM
+    const int grid = (int)(want < cap ? want : cap);
+    gather_rows<<<grid, 256, 0, st>>>((const uint4*)k, (const uint4*)v, idx, (uint4*)k_out,
+                                      (uint4*)v_out, s.seq_len, s.budget, vec_per_row, total);
+    return cudaGetLastError();
+}
+
+}  // namespace kvp
