@@ -20,8 +20,11 @@ Structure recipes (all bf16, all ~N(0,1) before structure is applied):
 * ``llama8b_32k_x32``: the same layer shape, 32 layers with independent seeds, B128.
 * ``long_128k_b70`` / ``long_128k_b10``: b1, 32/8 heads, d128, L131072, w32,
   B = floor(0.7 L) / floor(0.1 L); 4 outlier K/V channels x20, no rotation; 16 planted
-  needle keys per KV head at seeded positions j < L-w, each k_j = 24 sqrt(d) q / |q|^2
-  for a seeded window query q of that head's group, so its logit for q is 24.
+  needle keys per KV head at seeded positions j < L-w, each k_j = a sqrt(d) q / |q|^2
+  for a seeded window query q of that head's group, so its logit for q is a, with
+  a = max(24, 7 sigma_q). sigma_q = sqrt(sum_c q_c^2 s_c^2 / d) is the standard
+  deviation of q's logit against an ordinary key (channel scales s_c), so the needle
+  tops q's softmax row even when q leans on the x20 outlier channels.
 * ``gqa7_batched``: b8, 28/4 heads, d128, L16384, w64, B1024; a seed per sequence;
   4 outlier channels x20 in V only.
 
@@ -135,7 +138,8 @@ class Workload:
     outlier_scale: float = 20.0
     rope_base: float = 0.0
     needles: int = 0       # planted needle keys per KV head
-    needle_logit: float = 24.0
+    needle_logit: float = 24.0   # floor of a needle's logit for its query
+    needle_sigmas: float = 7.0   # ... and at least this many sigma_q
 
     @property
     def group(self) -> int:
@@ -216,6 +220,7 @@ def make_sequence(wl: Workload, layer: int = 0, seq: int = 0):
     if wl.needles:
         G = wl.group
         qf = bf16_to_f64(q)
+        ks = np.ones((hkv, d)) if kscale is None else kscale.astype(np.float64)
         for h in range(hkv):
             pos = _pick_distinct(seed, STREAM_NEEDLE, 4096 * h, wl.needles, L - w)
             needle_pos[h] = sorted(pos)
@@ -223,7 +228,9 @@ def make_sequence(wl: Workload, layer: int = 0, seq: int = 0):
                 r = int(draw_u64(seed, STREAM_NEEDLE, (1 << 24) + 64 * h + t, 1)[0] % np.uint64(G * w))
                 g, i = divmod(r, w)
                 qv = qf[h * G + g, i]
-                k[h, j] = round_bf16(wl.needle_logit * math.sqrt(d) * qv / float(qv @ qv))
+                sigma_q = math.sqrt(float(np.sum((qv * ks[h]) ** 2)) / d)
+                a = max(wl.needle_logit, wl.needle_sigmas * sigma_q)
+                k[h, j] = round_bf16(a * math.sqrt(d) * qv / float(qv @ qv))
     return q, k, v, needle_pos, kch, vch
 
 
