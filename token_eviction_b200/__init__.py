@@ -72,9 +72,10 @@ def _load():
 
 _lib = _load()
 
-# Kernel launches one layer's kvp_score + kvp_select + kvp_compact makes: log-sum-exp
-# pass, scoring pass, selection, gather.
-KERNELS_PER_LAYER = 4
+# Kernel launches one layer's kvp_score + kvp_select + kvp_compact makes: the fused
+# scoring kernel (both passes over K), the selection and the gather. kvp_score also
+# enqueues one small memset of its workspace counters.
+KERNELS_PER_LAYER = 3
 
 EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact", "kvp_status_string")
 

@@ -36,19 +36,26 @@ bool plan_of(const kvp_shape& s, Plan* p) {
     if (!shape_ok(s)) return false;
     p->G = s.hq / s.hkv;
     p->rows = p->G * s.window;
-    // Split L so that the log-sum-exp pass has about two CTAs per SM; splits are whole
-    // multiples of 128 keys. The split count does not depend on the device.
-    const int64_t units = (int64_t)s.batch * s.hkv;
-    const int tiles = (s.seq_len + 127) / 128;
-    int64_t want = (2 * 148 + units - 1) / units;
-    int nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(want, tiles));
-    int tiles_per_split = (tiles + nsplit - 1) / nsplit;
-    nsplit = (tiles + tiles_per_split - 1) / tiles_per_split;
-    p->nsplit = nsplit;
-    p->keys_per_split = tiles_per_split * 128;
+    const long long units = (long long)s.batch * s.hkv;
+    p->tiles_per_head = (s.seq_len + 127) / 128;
+    const long long T = units * p->tiles_per_head;
+    if (T > INT32_MAX) return false;
+    p->total_tiles = (int)T;
+    p->grid = (int)std::min<long long>(kPlanGrid, T);
+    int slots = 0;
+    for (long long h = 0; h < units; ++h) {
+        const long long f = h * p->tiles_per_head;
+        slots = std::max(slots, owner_of(f + p->tiles_per_head - 1, T, p->grid) -
+                                    owner_of(f, T, p->grid) + 1);
+    }
+    p->maxslots = slots;
     size_t off = 0;
+    p->off_done = off;
+    off += align_up((size_t)units * sizeof(uint32_t), 256);
+    p->off_err = off;
+    off += 256;
     p->off_part = off;
-    off += align_up((size_t)s.batch * s.hq * s.window * nsplit * sizeof(float2), 256);
+    off += align_up((size_t)s.batch * s.hq * s.window * slots * sizeof(float2), 256);
     p->off_select = off;
     off += 256;
     p->bytes = off;
@@ -78,11 +85,11 @@ extern "C" kvp_status kvp_score(const kvp_shape* shape, const uint16_t* q_win, c
         return KVP_ERR_ALIGN;
     if (!workspace || workspace_bytes < p.bytes) return KVP_ERR_WORKSPACE;
     if (!aligned16(workspace)) return KVP_ERR_ALIGN;
-    cudaStream_t st = (cudaStream_t)stream;
-    float2* part = (float2*)((char*)workspace + p.off_part);
-    if (launch_lse_partial(*shape, p, q_win, k, part, st) != cudaSuccess) return KVP_ERR_CUDA;
-    if (launch_score(*shape, p, q_win, k, v, part, score, s1, s2, st) != cudaSuccess)
+    if (launch_score(*shape, p, q_win, k, v, workspace, score, s1, s2, (cudaStream_t)stream) !=
+        cudaSuccess) {
+        cudaGetLastError();
         return KVP_ERR_CUDA;
+    }
     return KVP_OK;
 }
 

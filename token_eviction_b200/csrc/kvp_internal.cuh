@@ -12,27 +12,43 @@ namespace kvp {
 // one fp32 accumulator column per query row in tensor memory (512 columns per SM).
 constexpr int kMaxGroupRows = 512;
 
-// How a shape is cut into work: the split of L for the log-sum-exp pass and the
-// workspace layout. A pure function of the shape, so kvp_workspace_bytes, kvp_score
-// and kvp_select agree.
+// How a shape is cut into work: 128-key tiles of the flattened (sequence, KV head, key)
+// space dealt out in contiguous runs to the scoring kernel's CTAs, and the workspace
+// layout. A pure function of the shape, so kvp_workspace_bytes, kvp_score and
+// kvp_select agree.
 struct Plan {
-    int G;             // query heads per KV head
-    int rows;          // G * w: window queries per KV head
-    int nsplit;        // L-splits of the log-sum-exp pass
-    int keys_per_split;
-    size_t off_part;   // float2 (max, sum) partials [b*hq*w][nsplit], log2 domain
-    size_t off_select; // selection scratch
-    size_t bytes;      // total workspace
+    int G;               // query heads per KV head
+    int rows;            // G * w: window queries per KV head
+    int tiles_per_head;  // 128-key tiles per (sequence, KV head)
+    int total_tiles;     // over all (sequence, KV head)
+    int grid;            // CTAs of the scoring kernel (one per SM, at most one per tile)
+    int maxslots;        // partial-softmax slots per query row (CTAs touching one head)
+    size_t off_done;     // uint32 per (sequence, KV head): CTAs done with phase 0
+    size_t off_err;      // int: first device-side error code (0 = none)
+    size_t off_part;     // float2 (max, sum) partials [b*hq*w][maxslots], log2 domain
+    size_t off_select;   // selection scratch
+    size_t bytes;        // total workspace
 };
+
+// CTAs the scoring kernel is planned for (B200: 148 SMs); a device with fewer SMs runs
+// fewer, provided the workspace's slot count still covers every head.
+constexpr int kPlanGrid = 148;
 
 bool plan_of(const kvp_shape& s, Plan* p);
 
+// The CTA whose run holds tile t when T tiles are cut into `grid` contiguous runs
+// [floor(c T / grid), floor((c + 1) T / grid)).
+__host__ __device__ __forceinline__ int owner_of(long long t, long long T, long long grid) {
+    return (int)(((t + 1) * grid + T - 1) / T - 1);
+}
+__host__ __device__ __forceinline__ long long run_begin(long long c, long long T, long long grid) {
+    return c * T / grid;
+}
+
 // Launchers (each returns the launch's cudaError_t).
-cudaError_t launch_lse_partial(const kvp_shape& s, const Plan& p, const uint16_t* q,
-                               const uint16_t* k, float2* part, cudaStream_t st);
 cudaError_t launch_score(const kvp_shape& s, const Plan& p, const uint16_t* q, const uint16_t* k,
-                         const uint16_t* v, const float2* part, float* score, float* s1,
-                         float* s2, cudaStream_t st);
+                         const uint16_t* v, void* workspace, float* score, float* s1, float* s2,
+                         cudaStream_t st);
 cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score, int32_t* idx,
                           void* scratch, cudaStream_t st);
 cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t* v,
