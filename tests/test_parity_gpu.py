@@ -69,6 +69,9 @@ SMALL = {
     "short": synth.small("tiny", seq_len=50, window=10, budget=20),
     "window_is_all": synth.small("tiny", seq_len=16, window=16, budget=16),
     "one_tile_edge": synth.small("llama8b_32k", hq=4, hkv=1, seq_len=129, window=32, budget=64),
+    # more than 256 query rows per KV head: accumulators split across two TMEM stages
+    "split_ragged_g5": synth.small("llama8b_32k", hq=10, hkv=2, seq_len=900, window=56, budget=150),
+    "split_wide_window": synth.small("tiny", hq=2, hkv=2, head_dim=128, seq_len=700, window=300, budget=400),
 }
 
 
@@ -114,13 +117,18 @@ def test_gqa7_batched():
     check_layer(inp, gpu, *ora)
 
 
-@pytest.mark.parametrize("L,w,B", [(131072, 32, 91750), (32768, 32, 2048), (5000, 7, 4000), (4096, 64, 65)])
+@pytest.mark.parametrize("L,w,B", [(131072, 32, 91750), (131072, 32, 13107), (32768, 32, 2048),
+                                   (32768, 32, 128), (5000, 7, 4000), (4096, 64, 65), (70, 3, 9),
+                                   (350000, 16, 1000)])
 def test_select_exact_with_ties(L, w, B):
+    """Selection alone, on fp32 scores both sides share: the kept sets must be identical.
+    Rows: a large block of exact ties, zeros (and negative zeros), all-equal scores."""
     m = kvp()
     rng = np.random.default_rng(L + B)
     score = rng.random((3, L), dtype=np.float32) * np.float32(1e-3)
     score[0, : L // 2] = np.float32(5e-4)          # a large block of exact ties
     score[1, ::3] = 0.0
+    score[1, 1::7] = -0.0
     score[2] = np.float32(1.0)                      # every score equal
     score = score.reshape(1, 3, L)
     sh = m.make_shape(1, 3, 3, 128, L, w, B)

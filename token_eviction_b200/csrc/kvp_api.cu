@@ -29,6 +29,7 @@ static bool shape_ok(const kvp_shape& s) {
     if ((int64_t)s.batch * s.hkv > 65535) return false;  // grid y extent
     if ((int64_t)s.batch * s.hkv * s.seq_len > INT32_MAX) return false;
     if ((int64_t)s.batch * s.hq * s.window > INT32_MAX) return false;
+    if ((int64_t)s.batch * s.hkv * s.budget * 16 > INT32_MAX / 2) return false;  // gather pieces
     return true;
 }
 
@@ -48,7 +49,7 @@ bool plan_of(const kvp_shape& s, Plan* p) {
         slots = std::max(slots, owner_of(f + p->tiles_per_head - 1, T, p->grid) -
                                     owner_of(f, T, p->grid) + 1);
     }
-    p->maxslots = slots;
+    p->maxslots = slots * kSlotsPerCta;
     size_t off = 0;
     p->off_done = off;
     off += align_up((size_t)units * sizeof(uint32_t), 256);

@@ -34,6 +34,9 @@ struct Plan {
 // fewer, provided the workspace's slot count still covers every head.
 constexpr int kPlanGrid = 148;
 
+// Partial-softmax slots a CTA fills per KV head it touches (one per epilogue group).
+constexpr int kSlotsPerCta = 2;
+
 bool plan_of(const kvp_shape& s, Plan* p);
 
 // The CTA whose run holds tile t when T tiles are cut into `grid` contiguous runs

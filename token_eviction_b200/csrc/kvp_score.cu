@@ -14,19 +14,23 @@
 //     D[row, key] = Q_group[row] . K_tile[key] (M = query rows, N = 128 keys) into TMEM;
 //     the epilogue keeps, per query row, a running max m and sum l of 2^(t - m),
 //     t = logit * log2(e) / sqrt(d). At the end of each KV head in its run, a CTA
-//     publishes (m, l) per row into its slot and bumps the head's completion counter.
-//   phase 1 (scores): the same CTA sweeps the same tiles again. Before its first tile of
-//     a head it waits (bounded) until every CTA touching that head has published, then
-//     merges the slots into lse2 = M + log2(sum_s l_s 2^(m_s - M)) per row. Per tile,
-//     tcgen05 computes the transposed logits D[key, row] (M = 128 keys, N = G w rows), so
-//     each epilogue thread owns one key and sums 2^(t - lse2) over its row in TMEM
-//     columns with no cross-thread reduction; it reads the key's V row once from shared
-//     memory for S2 and writes S (and S1, S2 if asked).
+//     publishes (m, l) per row into its slots and bumps the head's completion counter.
+//   phase 1 (scores): the same CTA sweeps the same tiles again (K now mostly from L2).
+//     Before its first tile of a head it waits (bounded) until every CTA touching that
+//     head has published, then merges the slots into lse2 = M + log2(sum_s l_s 2^(m_s - M))
+//     per row. Per tile, tcgen05 computes the transposed logits D[key, row] (M = 128
+//     keys, N = G w rows), so each epilogue thread owns one key and sums 2^(t - lse2)
+//     over the row's TMEM columns with no cross-thread reduction; the key's V row is
+//     read once from shared memory for S2, and S (and S1, S2 if asked) is written.
 // Warp roles: warp 0 issues TMA loads (K ring, V ring, the group's query rows), warp 1
-// allocates TMEM and issues MMAs from one thread, warps 2-5 run the epilogue (one TMEM
-// lane quarter each). Every wait is bounded by a timer; a wait that gives up records an
-// error code in the workspace and the whole CTA unwinds without touching TMEM or
-// shared memory that may still be in use.
+// allocates TMEM and issues the MMAs from one thread, and two epilogue warpgroups
+// (warps 2-5 and 6-9, one TMEM lane quarter per warp) each own one of two TMEM
+// accumulator stages. When a tile's accumulator fits one stage (G w <= 256) the groups
+// take alternate tiles; otherwise every tile is split across both stages (query-row
+// halves in phase 0, column halves in phase 1) and the second group hands its partial
+// S1 to the first through shared memory.
+// Every wait is bounded by a timer; a wait that gives up records an error code in the
+// workspace and the CTA unwinds without touching TMEM or shared memory still in use.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -43,14 +47,17 @@ namespace kvp {
 
 namespace {
 
-constexpr int kTile = 128;                    // keys per tile
-constexpr int kThreads = 192;                 // 6 warps
-constexpr int kEpiThreads = 128;              // warps 2..5
+constexpr int kTile = 128;                        // keys per tile
+constexpr int kEpiGroups = 2;                     // epilogue warpgroups
+constexpr int kEpiThreads = 128 * kEpiGroups;
+constexpr int kThreads = 64 + kEpiThreads;        // + TMA warp + MMA warp
 constexpr int kMaxStages = 4;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kStageCols = 256;              // one accumulator stage per group
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s on any single wait
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kMinSmem = 116 * 1024;          // forces one CTA per SM (TMEM is taken whole)
+constexpr int kMinSmem = 116 * 1024;              // forces one CTA per SM (TMEM is taken whole)
+constexpr int kQBoxRows = 64;
 
 // error codes recorded in the workspace (first one wins)
 enum : int { kErrWaitTma = 1, kErrWaitMma = 2, kErrWaitEpi = 3, kErrWaitPeers = 4 };
@@ -58,18 +65,19 @@ enum : int { kErrWaitTma = 1, kErrWaitMma = 2, kErrWaitEpi = 3, kErrWaitPeers = 
 struct Params {
     int L, w, G, rows, hq, hkv, D;
     int mt;              // 128-row tiles covering the query group (phase 0 M tiles)
+    int mt0;             // split mode: M tiles in stage 0 (the rest in stage 1)
     int qrows;           // query rows staged in shared memory (rows rounded up to 64)
-    int n1, n2;          // phase 1 MMA N split of the group rows (n2 = 0: one MMA)
+    int n1, n2;          // phase 1 MMA N of the two column chunks (n2 = 0: one chunk)
+    int split;           // 0: groups alternate tiles; 1: every tile split over both stages
     int tiles_per_head, total_tiles, grid, maxslots;
     int nk, nv;          // K and V ring depths
-    int acc_stages, acc_stride;
     float scale2;        // log2(e) / sqrt(d)
     uint32_t q_bytes, k_bytes, v_bytes;
     uint32_t off_q, off_k, off_v, off_lse, off_bar;
     float* score;
     float* s1;
     float* s2;
-    float2* part;        // [b*hq*w][maxslots]
+    float2* part;        // [b*hq*w][maxslots]: (max, sum) in log2 units
     uint32_t* done;      // [b*hkv]
     int* err;
 };
@@ -78,17 +86,12 @@ struct SmemBars {
     uint64_t kfull[kMaxStages], kempty[kMaxStages];
     uint64_t vfull[kMaxStages], vempty[kMaxStages];
     uint64_t accfull[2], accempty[2];
+    uint64_t combfull[2], combempty[2];
     uint64_t qfull, qempty, fin;
-    uint64_t epi;        // epilogue-group rendezvous (128 arrivals per phase)
+    uint64_t epi;        // rendezvous of all epilogue threads
     uint32_t tmem_base;
     int abort_flag;
 };
-
-}  // namespace
-}  // namespace kvp
-
-namespace kvp {
-namespace {
 
 // Wait for phase `parity` of `bar`; false if the CTA is unwinding or the wait timed out
 // (then the first error code is recorded and the CTA told to unwind).
@@ -109,15 +112,8 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemB
     }
 }
 
-__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
-    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
-    __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
-    __nv_bfloat162 m = __hmax2(x, y);
-    return *reinterpret_cast<uint32_t*>(&m);
-}
-
-// Rendezvous of the 128 epilogue threads on an mbarrier, so that a thread that gives up
-// a wait can never leave the others blocked in a hardware barrier.
+// Rendezvous of all epilogue threads on an mbarrier, so that a thread that gives up a
+// wait can never leave the others blocked in a hardware barrier.
 __device__ __forceinline__ bool epi_sync(SmemBars* sb, uint32_t& phase, int* err) {
     ptx::mbar_arrive(&sb->epi);
     const bool ok = wait_phase(&sb->epi, phase, sb, err, kErrWaitEpi);
@@ -125,12 +121,18 @@ __device__ __forceinline__ bool epi_sync(SmemBars* sb, uint32_t& phase, int* err
     return ok;
 }
 
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
+    __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
+    __nv_bfloat162 m = __hmax2(x, y);
+    return *reinterpret_cast<uint32_t*>(&m);
+}
+
 // Segments of a CTA's run: maximal stretches of tiles within one KV head.
 struct RunIter {
     long long t, end;
     int tph;
     __device__ RunIter(long long b, long long e, int tiles_per_head) : t(b), end(e), tph(tiles_per_head) {}
-    // head of the next segment and its tile range [a, b)
     __device__ bool next(int& head, long long& a, long long& b) {
         if (t >= end) return false;
         head = (int)(t / tph);
@@ -141,6 +143,70 @@ struct RunIter {
     }
 };
 
+__device__ __forceinline__ float tree_max32(const float (&v)[32]) {
+    float m[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) m[e] = fmaxf(v[e], v[e + 16]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], m[e + 8]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m[e] = fmaxf(m[e], m[e + 4]);
+    return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
+}
+
+// Phase 0, one 32-key chunk of one query row: fold the chunk into the running (m, l).
+// `last` is the last key position the row sees; `key0` the chunk's first key.
+__device__ __forceinline__ void lse_chunk(float (&v)[32], bool full, int key0, int last,
+                                          float scale2, float& mrun, float& lrun) {
+    if (!full) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if (key0 + e > last) v[e] = -INFINITY;
+    }
+    const float cm = tree_max32(v);
+    if (cm == -INFINITY) return;
+    const float mn = fmaxf(mrun, cm * scale2);
+    float a0 = lrun * ptx::ex2(mrun - mn), a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+        a0 += ptx::ex2(fmaf(v[e + 0], scale2, -mn));
+        a1 += ptx::ex2(fmaf(v[e + 1], scale2, -mn));
+        a2 += ptx::ex2(fmaf(v[e + 2], scale2, -mn));
+        a3 += ptx::ex2(fmaf(v[e + 3], scale2, -mn));
+    }
+    lrun = (a0 + a1) + (a2 + a3);
+    mrun = mn;
+}
+
+// Phase 1, one 32-column chunk of one key: add 2^(t - lse2[n]) over the chunk's valid
+// query rows n = n0 + e (n < nend; inside the window, key offset jw <= n mod w).
+__device__ __forceinline__ void s1_chunk(const float (&v)[32], bool fast, int n0, int nend,
+                                         int jw, int w, const float* lse2, float scale2,
+                                         float& a0, float& a1, float& a2, float& a3) {
+    if (fast) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+            const float4 l4 = *(const float4*)(lse2 + n0 + e);
+            a0 += ptx::ex2(fmaf(v[e + 0], scale2, -l4.x));
+            a1 += ptx::ex2(fmaf(v[e + 1], scale2, -l4.y));
+            a2 += ptx::ex2(fmaf(v[e + 2], scale2, -l4.z));
+            a3 += ptx::ex2(fmaf(v[e + 3], scale2, -l4.w));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int n = n0 + e;
+            if (n < nend && jw <= n % w) a0 += ptx::ex2(fmaf(v[e], scale2, -lse2[n]));
+        }
+    }
+}
+
+}  // namespace
+}  // namespace kvp
+
+namespace kvp {
+namespace {
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -150,7 +216,8 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     uint8_t* Qs = smem + p.off_q;
     uint8_t* Ks = smem + p.off_k;
     uint8_t* Vs = smem + p.off_v;
-    float* lse2 = (float*)(smem + p.off_lse);
+    float* lse2 = (float*)(smem + p.off_lse);          // [512]
+    float* comb = lse2 + kMaxGroupRows;                 // [2][128] partial S1 handoff
     SmemBars* sb = (SmemBars*)(smem + p.off_bar);
 
     constexpr int kHalves = D / 64;                 // 128-byte swizzle rows per operand row
@@ -167,11 +234,13 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             ptx::mbar_init(&sb->kfull[s], 1);
             ptx::mbar_init(&sb->kempty[s], 1);
             ptx::mbar_init(&sb->vfull[s], 1);
-            ptx::mbar_init(&sb->vempty[s], kEpiThreads / 32);
+            ptx::mbar_init(&sb->vempty[s], 4);
         }
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&sb->accfull[s], 1);
-            ptx::mbar_init(&sb->accempty[s], kEpiThreads / 32);
+            ptx::mbar_init(&sb->accempty[s], 4);
+            ptx::mbar_init(&sb->combfull[s], 4);
+            ptx::mbar_init(&sb->combempty[s], 4);
         }
         ptx::mbar_init(&sb->qfull, 1);
         ptx::mbar_init(&sb->qempty, 1);
@@ -215,7 +284,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         if (qgen > 0 && !(ok = wait_phase(&sb->qempty, (qgen - 1) & 1, sb, p.err, kErrWaitTma))) break;
                         ptx::mbar_arrive_expect_tx(&sb->qfull, p.q_bytes);
                         const int r0 = group_row0(head);
-                        for (int rb = 0; rb < p.qrows; rb += 64)
+                        for (int rb = 0; rb < p.qrows; rb += kQBoxRows)
                             for (int c = 0; c < kHalves; ++c)
                                 ptx::tma_load_2d(Qs + c * qhalf + rb * 128, &qmap, &sb->qfull,
                                                  c * 64, r0 + rb, pol_keep);
@@ -271,32 +340,41 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     }
                     for (long long t = a; t < b; ++t) {
                         const int s = kit % p.nk;
-                        const int sa = ait % p.acc_stages;
                         if (!(ok = wait_phase(&sb->kfull[s], (kit / p.nk) & 1, sb, p.err, kErrWaitMma))) break;
-                        if (!(ok = wait_phase(&sb->accempty[sa], ((ait / p.acc_stages) & 1) ^ 1, sb, p.err, kErrWaitMma))) break;
-                        ptx::tc_fence_after();
-                        const uint32_t d0 = tmem + (uint32_t)(sa * p.acc_stride);
                         const uint32_t kbase = k_addr + s * kstage;
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const int c = ks >> 2, kk = ks & 3;
-                            const uint32_t koff = kbase + c * kHalfTile + kk * 32;
-                            const uint32_t qoff = q_addr + c * qhalf + kk * 32;
-                            if (phase == 0) {
-                                for (int m = 0; m < p.mt; ++m)
-                                    ptx::mma_bf16_ss(d0 + m * kTile,
-                                                     ptx::sw128_kmajor_desc(qoff + m * kHalfTile),
-                                                     ptx::sw128_kmajor_desc(koff), idesc0, ks > 0);
-                            } else {
-                                const uint64_t adesc = ptx::sw128_kmajor_desc(koff);
-                                ptx::mma_bf16_ss(d0, adesc, ptx::sw128_kmajor_desc(qoff), idesc1a, ks > 0);
-                                if (p.n2 > 0)
-                                    ptx::mma_bf16_ss(d0 + p.n1, adesc,
-                                                     ptx::sw128_kmajor_desc(qoff + p.n1 * 128), idesc1b,
-                                                     ks > 0);
+                        // stages written for this tile: one (alternating) or both (split)
+                        const int st_lo = p.split ? 0 : (ait & 1);
+                        const int st_hi = p.split ? 1 : (ait & 1);
+                        const uint32_t use_parity = p.split ? (ait & 1) : ((ait >> 1) & 1);
+                        for (int st = st_lo; st <= st_hi && ok; ++st) {
+                            if (!(ok = wait_phase(&sb->accempty[st], use_parity ^ 1, sb, p.err, kErrWaitMma))) break;
+                            ptx::tc_fence_after();
+                            const uint32_t d0 = tmem + (uint32_t)st * kStageCols;
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const int c = ks >> 2, kk = ks & 3;
+                                const uint32_t koff = kbase + c * kHalfTile + kk * 32;
+                                const uint32_t qoff = q_addr + c * qhalf + kk * 32;
+                                if (phase == 0) {
+                                    const int mlo = p.split ? st * p.mt0 : 0;
+                                    const int mhi = p.split ? (st ? p.mt : p.mt0) : p.mt;
+                                    for (int m = mlo; m < mhi; ++m)
+                                        ptx::mma_bf16_ss(d0 + (m - mlo) * kTile,
+                                                         ptx::sw128_kmajor_desc(qoff + m * kHalfTile),
+                                                         ptx::sw128_kmajor_desc(koff), idesc0, ks > 0);
+                                } else {
+                                    const uint64_t adesc = ptx::sw128_kmajor_desc(koff);
+                                    if (!p.split || st == 0)
+                                        ptx::mma_bf16_ss(d0, adesc, ptx::sw128_kmajor_desc(qoff), idesc1a, ks > 0);
+                                    if (p.n2 > 0 && (!p.split || st == 1))
+                                        ptx::mma_bf16_ss(d0 + (p.split ? 0 : p.n1), adesc,
+                                                         ptx::sw128_kmajor_desc(qoff + p.n1 * 128),
+                                                         idesc1b, ks > 0);
+                                }
                             }
+                            ptx::mma_commit(&sb->accfull[st]);
                         }
+                        if (!ok) break;
                         ptx::mma_commit(&sb->kempty[s]);
-                        ptx::mma_commit(&sb->accfull[sa]);
                         ++kit;
                         ++ait;
                     }
@@ -321,12 +399,15 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - 64;                  // 0..127
+        const int et = threadIdx.x - 64;                  // 0 .. kEpiThreads-1
+        const int wg = et >> 7;                           // epilogue group = TMEM stage
         const int quarter = warp & 3;                     // TMEM lane quarter of this warp
-        const int lrow = quarter * 32 + lane;             // lane owned: row (phase 0) or key (phase 1)
-        const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
+        const int lrow = quarter * 32 + lane;             // lane: query row (phase 0) / key (phase 1)
+        const uint32_t tstage = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)wg * kStageCols;
         const int window0 = p.L - p.w;                    // first window position
-        int ait = 0, vit = 0;
+        const int mlo = p.split ? wg * p.mt0 : 0;         // phase 0 M tiles of this group
+        const int mhi = p.split ? (wg ? p.mt : p.mt0) : p.mt;
+        int ait = 0;
         uint32_t epi_phase = 0;
         bool ok = true;
         // ---- phase 0: per-row running max and sum over this CTA's keys of each head
@@ -337,56 +418,54 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             while (ok && it.next(head, a, b)) {
                 float mrun[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 float lrun[4] = {0.f, 0.f, 0.f, 0.f};
-                for (long long t = a; t < b && ok; ++t) {
-                    const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
-                    const int sa = ait % p.acc_stages;
-                    if (!(ok = wait_phase(&sb->accfull[sa], (ait / p.acc_stages) & 1, sb, p.err, kErrWaitEpi))) break;
+                for (long long t = a; t < b && ok; ++t, ++ait) {
+                    if (!p.split && (ait & 1) != wg) continue;       // the other group's tile
+                    const uint32_t parity = p.split ? (ait & 1) : ((ait >> 1) & 1);
+                    if (!(ok = wait_phase(&sb->accfull[wg], parity, sb, p.err, kErrWaitEpi))) break;
                     ptx::tc_fence_after();
+                    const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
                     const bool full = key0 + kTile - 1 <= window0;   // every row sees every key
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        if (m >= p.mt) break;                        // uniform across the CTA
+                        if (m < mlo || m >= mhi) continue;           // uniform across the group
                         const int r = m * kTile + lrow;
                         const int last = window0 + (r % p.w);        // last key row r sees
-#pragma unroll 1
-                        for (int ch = 0; ch < kTile / 32; ++ch) {
-                            float v[32];
-                            __syncwarp();
-                            ptx::tmem_ld_32x32b_x32(tmem + lane_bits + sa * p.acc_stride + m * kTile + ch * 32, v);
-                            ptx::tmem_ld_wait();
-                            if (!full) {
-#pragma unroll
-                                for (int e = 0; e < 32; ++e)
-                                    if (key0 + ch * 32 + e > last) v[e] = -INFINITY;
-                            }
-                            float cm = v[0];
-#pragma unroll
-                            for (int e = 1; e < 32; ++e) cm = fmaxf(cm, v[e]);
-                            if (cm != -INFINITY) {
-                                const float mn = fmaxf(mrun[m], cm * p.scale2);
-                                float acc = lrun[m] * ptx::ex2(mrun[m] - mn);
-#pragma unroll
-                                for (int e = 0; e < 32; ++e) acc += ptx::ex2(fmaf(v[e], p.scale2, -mn));
-                                lrun[m] = acc;
-                                mrun[m] = mn;
-                            }
-                        }
+                        const uint32_t tb = tstage + (uint32_t)(m - mlo) * kTile;
+                        float x[32], y[32];
+                        __syncwarp();
+                        ptx::tmem_ld_32x32b_x32(tb, x);
+                        ptx::tmem_ld_wait(x);
+                        __syncwarp();
+                        ptx::tmem_ld_32x32b_x32(tb + 32, y);
+                        lse_chunk(x, full, key0, last, p.scale2, mrun[m], lrun[m]);
+                        ptx::tmem_ld_wait(y);
+                        __syncwarp();
+                        ptx::tmem_ld_32x32b_x32(tb + 64, x);
+                        lse_chunk(y, full, key0 + 32, last, p.scale2, mrun[m], lrun[m]);
+                        ptx::tmem_ld_wait(x);
+                        __syncwarp();
+                        ptx::tmem_ld_32x32b_x32(tb + 96, y);
+                        lse_chunk(x, full, key0 + 64, last, p.scale2, mrun[m], lrun[m]);
+                        ptx::tmem_ld_wait(y);
+                        lse_chunk(y, full, key0 + 96, last, p.scale2, mrun[m], lrun[m]);
                     }
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[sa]);
-                    ++ait;
+                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[wg]);
                 }
                 if (!ok) break;
-                // publish this CTA's partials for `head`
+                // publish this group's partials for `head` into its own slot
                 const long long first = (long long)head * p.tiles_per_head;
-                const int slot = (int)blockIdx.x - owner_of(first, T, p.grid);
+                const int slot = ((int)blockIdx.x - owner_of(first, T, p.grid)) * kSlotsPerCta + wg;
                 const int r0 = group_row0(head);
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     const int r = m * kTile + lrow;
-                    if (m < p.mt && r < p.rows)
-                        p.part[(size_t)(r0 + r) * p.maxslots + slot] = make_float2(mrun[m], lrun[m]);
+                    if (m < p.mt && r < p.rows) {
+                        const bool mine = m >= mlo && m < mhi;
+                        p.part[(size_t)(r0 + r) * p.maxslots + slot] =
+                            mine ? make_float2(mrun[m], lrun[m]) : make_float2(-INFINITY, 0.f);
+                    }
                 }
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
                 if (et == 0) {
@@ -400,10 +479,11 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             RunIter it(t0, t1, p.tiles_per_head);
             int head;
             long long a, b;
+            int pt = 0;                                   // phase 1 tile counter (V ring, handoff)
             while (ok && it.next(head, a, b)) {
                 const long long first = (long long)head * p.tiles_per_head;
                 const int touch = owner_of(first + p.tiles_per_head - 1, T, p.grid) - owner_of(first, T, p.grid) + 1;
-                // previous head's lse2 no longer in use
+                // the previous head's lse2 is no longer in use
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
                 if (et == 0) {
                     const uint64_t ts = ptx::globaltimer_ns();
@@ -423,78 +503,103 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     break;
                 }
                 const int r0 = group_row0(head);
+                const int nslots = touch * kSlotsPerCta;
                 for (int r = et; r < p.rows; r += kEpiThreads) {
                     const float2* pr = p.part + (size_t)(r0 + r) * p.maxslots;
                     float M = -INFINITY;
-                    for (int s = 0; s < touch; ++s) M = fmaxf(M, __ldcg(&pr[s].x));
+                    for (int s = 0; s < nslots; ++s) M = fmaxf(M, __ldcg(&pr[s].x));
                     float sum = 0.f;
-                    for (int s = 0; s < touch; ++s) {
+                    for (int s = 0; s < nslots; ++s) {
                         const float2 ml = __ldcg(pr + s);
                         if (ml.x != -INFINITY) sum += ml.y * ptx::ex2(ml.x - M);
                     }
                     lse2[r] = M + __log2f(sum);
                 }
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
-                for (long long t = a; t < b && ok; ++t) {
+                for (long long t = a; t < b && ok; ++t, ++ait, ++pt) {
+                    const bool mine = p.split || (ait & 1) == wg;
+                    if (!mine) continue;
+                    const bool reads_v = !p.split || wg == 0;
                     const int key0 = (int)(t - first) * kTile;
                     const int j = key0 + lrow;
-                    // S2: max |V[j, :]| from the staged tile (16-byte pieces in a rotated
-                    // order per lane, which keeps the shared-memory reads conflict-free)
-                    const int sv = vit % p.nv;
-                    if (!(ok = wait_phase(&sb->vfull[sv], (vit / p.nv) & 1, sb, p.err, kErrWaitEpi))) break;
-                    const uint4* vrow = (const uint4*)(Vs + sv * vstage + lrow * (D * 2));
-                    constexpr int kPieces = D * 2 / 16;
-                    uint32_t mx = 0;
+                    float s2v = 0.f;
+                    if (reads_v) {
+                        // S2: max |V[j, :]| from the staged tile, 16-byte pieces in a
+                        // rotated order per lane (conflict-free shared-memory reads)
+                        const int sv = pt % p.nv;
+                        if (!(ok = wait_phase(&sb->vfull[sv], (pt / p.nv) & 1, sb, p.err, kErrWaitEpi))) break;
+                        const uint4* vrow = (const uint4*)(Vs + sv * vstage + lrow * (D * 2));
+                        constexpr int kPieces = D * 2 / 16;
+                        uint32_t mx = 0;
 #pragma unroll
-                    for (int c = 0; c < kPieces; ++c) {
-                        const uint4 x = vrow[(c + lane) & (kPieces - 1)];
-                        mx = bf16x2_absmax(mx, x.x & 0x7FFF7FFFu);
-                        mx = bf16x2_absmax(mx, x.y & 0x7FFF7FFFu);
-                        mx = bf16x2_absmax(mx, x.z & 0x7FFF7FFFu);
-                        mx = bf16x2_absmax(mx, x.w & 0x7FFF7FFFu);
+                        for (int c = 0; c < kPieces; ++c) {
+                            const uint4 x = vrow[(c + lane) & (kPieces - 1)];
+                            mx = bf16x2_absmax(mx, x.x & 0x7FFF7FFFu);
+                            mx = bf16x2_absmax(mx, x.y & 0x7FFF7FFFu);
+                            mx = bf16x2_absmax(mx, x.z & 0x7FFF7FFFu);
+                            mx = bf16x2_absmax(mx, x.w & 0x7FFF7FFFu);
+                        }
+                        s2v = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&sb->vempty[sv]);
                     }
-                    const float s2v = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&sb->vempty[sv]);
-                    ++vit;
-                    // S1: sum over the group's window queries of 2^(t - lse2)
-                    const int sa = ait % p.acc_stages;
-                    if (!(ok = wait_phase(&sb->accfull[sa], (ait / p.acc_stages) & 1, sb, p.err, kErrWaitEpi))) break;
+                    // S1 over this group's columns
+                    const uint32_t parity = p.split ? (ait & 1) : ((ait >> 1) & 1);
+                    if (!(ok = wait_phase(&sb->accfull[wg], parity, sb, p.err, kErrWaitEpi))) break;
                     ptx::tc_fence_after();
                     const bool full = key0 + kTile - 1 <= window0;
-                    const int jw = j - window0;       // > 0 only inside the window
-                    float acc = 0.f;
-                    for (int n0 = 0; n0 < p.rows; n0 += 32) {
-                        float v[32];
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tmem + lane_bits + sa * p.acc_stride + n0, v);
-                        ptx::tmem_ld_wait();
-                        if (full && n0 + 32 <= p.rows) {
-#pragma unroll
-                            for (int e = 0; e < 32; e += 4) {
-                                const float4 l4 = *(const float4*)(lse2 + n0 + e);
-                                acc += ptx::ex2(fmaf(v[e + 0], p.scale2, -l4.x));
-                                acc += ptx::ex2(fmaf(v[e + 1], p.scale2, -l4.y));
-                                acc += ptx::ex2(fmaf(v[e + 2], p.scale2, -l4.z));
-                                acc += ptx::ex2(fmaf(v[e + 3], p.scale2, -l4.w));
+                    const int jw = j - window0;                     // > 0 only inside the window
+                    const int col0 = (p.split && wg == 1) ? p.n1 : 0;        // first query row
+                    const int ncols = p.split ? (wg == 0 ? p.n1 : p.rows - p.n1) : p.rows;
+                    const int nch = (ncols + 31) >> 5;
+                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                    float x[32], y[32];
+                    __syncwarp();
+                    ptx::tmem_ld_32x32b_x32(tstage, x);
+                    ptx::tmem_ld_wait(x);
+                    for (int c = 0; c < nch; c += 2) {
+                        const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
+                        if (has1) {
+                            __syncwarp();
+                            ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
+                        }
+                        s1_chunk(x, full && (c + 1) * 32 <= ncols, col0 + c * 32, col0 + ncols, jw, p.w,
+                                 lse2, p.scale2, a0, a1, a2, a3);
+                        if (has1) {
+                            ptx::tmem_ld_wait(y);
+                            if (has2) {
+                                __syncwarp();
+                                ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
                             }
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const int n = n0 + e;
-                                if (n < p.rows && jw <= n % p.w)
-                                    acc += ptx::ex2(fmaf(v[e], p.scale2, -lse2[n]));
-                            }
+                            s1_chunk(y, full && (c + 2) * 32 <= ncols, col0 + (c + 1) * 32, col0 + ncols, jw,
+                                     p.w, lse2, p.scale2, a0, a1, a2, a3);
+                            if (has2) ptx::tmem_ld_wait(x);
                         }
                     }
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[sa]);
-                    ++ait;
+                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[wg]);
+                    float s1v = (a0 + a1) + (a2 + a3);
+                    if (p.split) {
+                        // hand the second group's partial to the first
+                        const int cb = pt & 1;
+                        const uint32_t cpar = (pt >> 1) & 1;
+                        if (wg == 1) {
+                            if (!(ok = wait_phase(&sb->combempty[cb], cpar ^ 1, sb, p.err, kErrWaitEpi))) break;
+                            comb[cb * kTile + lrow] = s1v;
+                            __syncwarp();
+                            if (lane == 0) ptx::mbar_arrive(&sb->combfull[cb]);
+                            continue;
+                        }
+                        if (!(ok = wait_phase(&sb->combfull[cb], cpar, sb, p.err, kErrWaitEpi))) break;
+                        s1v += comb[cb * kTile + lrow];
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&sb->combempty[cb]);
+                    }
                     if (j < p.L) {
                         const size_t o = (size_t)head * p.L + j;
-                        p.score[o] = acc * s2v;
-                        if (p.s1) p.s1[o] = acc;
+                        p.score[o] = s1v * s2v;
+                        if (p.s1) p.s1[o] = s1v;
                         if (p.s2) p.s2[o] = s2v;
                     }
                 }
@@ -544,8 +649,6 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* di
     return r == CUDA_SUCCESS;
 }
 
-constexpr int kQBoxRows = 64;
-
 struct Launch {
     Params p;
     int grid;
@@ -571,6 +674,8 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
         p.n1 = (npad / 2 + 15) / 16 * 16;
         p.n2 = npad - p.n1;
     }
+    p.split = plan.rows > (int)kStageCols ? 1 : 0;
+    p.mt0 = (p.mt + 1) / 2;
     p.tiles_per_head = plan.tiles_per_head;
     p.total_tiles = plan.total_tiles;
     p.grid = std::min(plan.grid, sms);
@@ -582,7 +687,7 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
             const long long f = (long long)h * p.tiles_per_head;
             need = std::max(need, owner_of(f + p.tiles_per_head - 1, T, p.grid) - owner_of(f, T, p.grid) + 1);
         }
-        if (need > plan.maxslots) return false;
+        if (need * kSlotsPerCta > plan.maxslots) return false;
     }
     p.maxslots = plan.maxslots;
     p.scale2 = 1.4426950408889634f / sqrtf((float)D);
@@ -593,18 +698,10 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.q_bytes = qbytes;
     p.k_bytes = tile_bytes;
     p.v_bytes = tile_bytes;
-    // TMEM: two accumulator stages of 256 columns when both phases fit, else one of 512
-    const int cols0 = p.mt * kTile, cols1 = (npad + 31) / 32 * 32;
-    if (cols0 <= 256 && cols1 <= 256) {
-        p.acc_stages = 2;
-        p.acc_stride = 256;
-    } else {
-        p.acc_stages = 1;
-        p.acc_stride = 512;
-    }
-    // shared memory: Q | K ring | V ring | lse2 | barriers (+1 KB to align the base)
+    // shared memory: Q | K ring | V ring | lse2 + handoff | barriers (+1 KB to align the base)
     const int choices[5][2] = {{4, 2}, {3, 2}, {2, 2}, {3, 1}, {2, 1}};
-    const size_t fixed = 2048 + 256 + 1024;
+    const size_t lse_bytes = (kMaxGroupRows + 2 * kTile) * sizeof(float);
+    const size_t fixed = lse_bytes + 256 + 1024;
     size_t total = 0;
     bool fit = false;
     for (auto& c : choices) {
@@ -621,7 +718,7 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.off_k = qbytes;
     p.off_v = p.off_k + p.nk * tile_bytes;
     p.off_lse = p.off_v + p.nv * tile_bytes;
-    p.off_bar = p.off_lse + 2048;
+    p.off_bar = p.off_lse + (uint32_t)lse_bytes;
     static_assert(sizeof(SmemBars) <= 256, "barrier block");
     L->grid = p.grid;
     L->smem = std::max(total, (size_t)kMinSmem);

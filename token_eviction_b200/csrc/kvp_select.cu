@@ -5,19 +5,32 @@
 // [L - w, L) and the B - w highest scores among [0, L - w); equal scores go to the
 // lower position; the list is written in ascending position order.
 //
-// One CTA per row. A radix select over an order-preserving 32-bit image of the fp32
-// scores finds the exact threshold value T (the (B - w)-th largest) in four 8-bit
-// passes, and how many elements equal to T are still needed; an ordered pass then
-// emits, in position order, every element above T and the first needed ones equal to
-// T, with block-wide prefix sums giving each its output slot.
+// One thread-block cluster of kCl CTAs per row. Each CTA holds a contiguous slice of
+// the row's candidates in shared memory as order-preserving 32-bit keys (the fp32 bit
+// pattern with the sign handled so that unsigned order equals numeric order).
+// A radix select over the keys finds the exact threshold T (the (B - w)-th largest key)
+// in three passes of 11, 11 and 10 bits: every CTA histograms its slice (only keys that
+// match the prefix found so far), adds its histogram into the leader CTA's through
+// distributed shared memory, and the leader picks the digit where the count from the top
+// reaches the number still needed. The emission then writes, in position order, every key
+// above T and the first keys equal to T (as many as still needed); each warp's output
+// offset comes from counts exchanged across the cluster. Only cluster and block
+// barriers are used: every CTA takes the same steps, so none can wait forever.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include "kvp_internal.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace kvp {
 namespace {
 
-constexpr int kSelectThreads = 1024;
+constexpr int kCl = 8;              // CTAs per row (portable cluster size)
+constexpr int kSelThreads = 1024;
+constexpr int kWarps = kSelThreads / 32;
+constexpr int kBins = 2048;
+constexpr int kSliceCap = 40960;    // keys per CTA held in shared memory
 
 // Order-preserving map of fp32 bits to uint32 (-0 is treated as +0; NaN unsupported).
 __device__ __forceinline__ uint32_t order_key(uint32_t bits) {
@@ -25,8 +38,18 @@ __device__ __forceinline__ uint32_t order_key(uint32_t bits) {
     return (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
 }
 
-// Exclusive block-wide prefix sum of `x` over kSelectThreads threads; *total gets the sum.
-__device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int* total) {
+struct SelShared {
+    unsigned hist[kBins];      // this CTA's histogram
+    unsigned merged[kBins];    // leader only: the cluster's histogram
+    unsigned digit, krem;      // leader only: result of the current pass
+    unsigned cta_gt[kCl], cta_eq[kCl];  // leader only: per-CTA counts for the emission
+    unsigned warp_gt[kWarps], warp_eq[kWarps];
+    unsigned warp_sel_off[kWarps], warp_eq_off[kWarps];
+    int scan[kWarps + 1];
+};
+
+// Exclusive prefix sum over the block (kSelThreads threads); returns this thread's.
+__device__ __forceinline__ int block_exclusive_scan(int x, int* ws) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int inc = x;
 #pragma unroll
@@ -34,91 +57,172 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int* 
         const int y = __shfl_up_sync(0xffffffffu, inc, o);
         if (lane >= o) inc += y;
     }
-    if (lane == 31) warp_sums[warp] = inc;
+    if (lane == 31) ws[warp] = inc;
     __syncthreads();
     if (warp == 0) {
-        int ws = warp_sums[lane];
-        int wi = ws;
+        const int v = ws[lane];
+        int wi = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, wi, o);
             if (lane >= o) wi += y;
         }
-        warp_sums[lane] = wi - ws;  // exclusive prefix of warp totals
-        if (lane == 31) warp_sums[32] = wi;
+        ws[lane] = wi - v;
     }
     __syncthreads();
-    const int result = warp_sums[warp] + inc - x;
-    *total = warp_sums[32];
-    __syncthreads();  // warp_sums is reused by the next call
-    return result;
+    const int r = ws[warp] + inc - x;
+    __syncthreads();
+    return r;
 }
 
-__global__ void __launch_bounds__(kSelectThreads) select_topk_rows(const float* __restrict__ score,
-                                                                   int32_t* __restrict__ idx,
-                                                                   int L, int w, int B) {
-    __shared__ unsigned hist[256];
-    __shared__ int warp_sums[33];
-    __shared__ unsigned s_digit, s_krem;
-    const int row = blockIdx.x;
-    const uint32_t* key = reinterpret_cast<const uint32_t*>(score + (size_t)row * L);
+template <bool kInSmem>
+__global__ void __launch_bounds__(kSelThreads, 1)
+select_cluster(const float* __restrict__ score, int32_t* __restrict__ idx, int L, int w, int B,
+               int slice) {
+    extern __shared__ uint32_t keys[];   // [slice] when kInSmem
+    __shared__ SelShared sh;
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned rank = cluster.block_rank();
+    const int row = blockIdx.x / kCl;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = L - w, kk = B - w;
+    const uint32_t* rowbits = reinterpret_cast<const uint32_t*>(score + (size_t)row * L);
     int32_t* out = idx + (size_t)row * B;
-    const int n = L - w;   // candidates
-    const int kk = B - w;  // to keep among them
-    const int tid = threadIdx.x;
 
-    for (int t = tid; t < w; t += blockDim.x) out[kk + t] = n + t;
-    if (kk == 0) return;
+    if (rank == 0)
+        for (int t = tid; t < w; t += kSelThreads) out[kk + t] = n + t;
+    if (kk == 0) return;                  // same decision in every CTA of the cluster
     if (kk == n) {
-        for (int t = tid; t < n; t += blockDim.x) out[t] = t;
+        for (int t = (int)rank * kSelThreads + tid; t < n; t += kCl * kSelThreads) out[t] = t;
         return;
     }
 
-    // Radix select of the kk-th largest order key, 8 bits at a time from the top.
+    const int lo = min(n, (int)rank * slice), hi = min(n, lo + slice);
+    auto key_at = [&](int j) -> uint32_t {  // j in [lo, hi)
+        if (kInSmem) return keys[j - lo];
+        return order_key(__ldg(rowbits + j));
+    };
+    if (kInSmem) {
+        for (int j = lo + tid; j < hi; j += kSelThreads) keys[j - lo] = order_key(__ldg(rowbits + j));
+    }
+    SelShared* leader = cluster.map_shared_rank(&sh, 0);
+
+    // ---- radix select: 11 + 11 + 10 bits from the top
     uint32_t prefix = 0, mask = 0, krem = (uint32_t)kk;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int t = tid; t < 256; t += blockDim.x) hist[t] = 0;
-        __syncthreads();
-        for (int j = tid; j < n; j += blockDim.x) {
-            const uint32_t u = order_key(__ldg(key + j));
-            if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    const int shifts[3] = {21, 10, 0};
+    const uint32_t widths[3] = {2047u, 2047u, 1023u};
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = shifts[pass];
+        const uint32_t dmask = widths[pass];
+        for (int b = tid; b < kBins; b += kSelThreads) {
+            sh.hist[b] = 0;
+            if (rank == 0) sh.merged[b] = 0;
+        }
+        cluster.sync();                    // merged histogram cleared (and keys staged)
+        for (int j = lo + tid; j < hi; j += kSelThreads) {
+            const uint32_t u = key_at(j);
+            if ((u & mask) == prefix) atomicAdd(&sh.hist[(u >> shift) & dmask], 1u);
         }
         __syncthreads();
-        if (tid == 0) {
-            uint32_t cum = 0;
-            for (int dg = 255; dg >= 0; --dg) {
-                const uint32_t c = hist[dg];
-                if (cum + c >= krem) {
-                    s_digit = (uint32_t)dg;
-                    s_krem = krem - cum;
-                    break;
-                }
-                cum += c;
+        for (int b = tid; b < kBins; b += kSelThreads)
+            if (sh.hist[b]) atomicAdd(&leader->merged[b], sh.hist[b]);
+        cluster.sync();                    // merged histogram complete
+        if (rank == 0) {
+            // thread t holds the bin pair (2047 - 2t, 2046 - 2t): count of all higher bins
+            const int bh = kBins - 1 - 2 * tid, bl = bh - 1;
+            const unsigned ch = sh.merged[bh], cl = sh.merged[bl];
+            const unsigned above = (unsigned)block_exclusive_scan((int)(ch + cl), sh.scan);
+            if (above < krem && krem <= above + ch) {
+                sh.digit = (unsigned)bh;
+                sh.krem = krem - above;
+            } else if (above + ch < krem && krem <= above + ch + cl) {
+                sh.digit = (unsigned)bl;
+                sh.krem = krem - above - ch;
             }
         }
-        __syncthreads();
-        prefix |= s_digit << shift;
-        mask |= 255u << shift;
-        krem = s_krem;
-        __syncthreads();
+        cluster.sync();                    // digit published
+        const unsigned dg = leader->digit, kr = leader->krem;
+        prefix |= dg << shift;
+        mask |= dmask << shift;
+        krem = kr;
     }
-    const uint32_t T = prefix;      // order key of the kk-th largest score
-    const int need_eq = (int)krem;  // how many keys equal to T are kept (lowest positions)
+    const uint32_t T = prefix;             // key of the (B - w)-th largest score
+    const unsigned need_eq = krem;         // keys equal to T that are kept (lowest positions)
 
-    int carry_eq = 0, carry_sel = 0;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int j = base + tid;
-        const uint32_t u = j < n ? order_key(__ldg(key + j)) : 0u;
-        const int gt = (j < n && u > T) ? 1 : 0;
-        const int eq = (j < n && u == T) ? 1 : 0;
-        int tot_eq, tot_sel;
-        const int eq_rank = carry_eq + block_exclusive_scan(eq, warp_sums, &tot_eq);
-        const int sel = (gt || (eq && eq_rank < need_eq)) ? 1 : 0;
-        const int slot = carry_sel + block_exclusive_scan(sel, warp_sums, &tot_sel);
-        if (sel) out[slot] = j;
-        carry_eq += tot_eq;
-        carry_sel += tot_sel;
+    // ---- ordered emission: warp w covers a contiguous stretch of this CTA's slice
+    const int span = hi - lo;
+    const int per_warp = ((span + kWarps - 1) / kWarps + 31) / 32 * 32;
+    const int wlo = lo + warp * per_warp, whi = min(hi, wlo + per_warp);
+    unsigned cgt = 0, ceq = 0;
+    for (int j0 = wlo; j0 < whi; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t u = j < whi ? key_at(j) : 0u;
+        cgt += __popc(__ballot_sync(0xffffffffu, j < whi && u > T));
+        ceq += __popc(__ballot_sync(0xffffffffu, j < whi && u == T));
     }
+    if (lane == 0) {
+        sh.warp_gt[warp] = cgt;
+        sh.warp_eq[warp] = ceq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        unsigned g = sh.warp_gt[lane], e = sh.warp_eq[lane];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            e += __shfl_xor_sync(0xffffffffu, e, o);
+        }
+        if (lane == 0) {
+            leader->cta_gt[rank] = g;
+            leader->cta_eq[rank] = e;
+        }
+    }
+    cluster.sync();                        // every CTA's counts at the leader
+    if (warp == 0) {
+        // offsets of this CTA: equal keys and kept keys in all lower-ranked CTAs
+        unsigned eq_before = 0, sel_before = 0;
+        for (unsigned r = 0; r < rank; ++r) {
+            const unsigned g = leader->cta_gt[r], e = leader->cta_eq[r];
+            const unsigned take = eq_before >= need_eq ? 0u : min(e, need_eq - eq_before);
+            sel_before += g + take;
+            eq_before += e;
+        }
+        // then per warp, in position order
+        const unsigned g = sh.warp_gt[lane], e = sh.warp_eq[lane];
+        unsigned einc = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, einc, o);
+            if (lane >= o) einc += y;
+        }
+        const unsigned weq_before = eq_before + einc - e;
+        const unsigned take = weq_before >= need_eq ? 0u : min(e, need_eq - weq_before);
+        const unsigned s = g + take;
+        unsigned sinc = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, sinc, o);
+            if (lane >= o) sinc += y;
+        }
+        sh.warp_sel_off[lane] = sel_before + sinc - s;
+        sh.warp_eq_off[lane] = weq_before;
+    }
+    __syncthreads();
+    unsigned pos = sh.warp_sel_off[warp], eq_run = sh.warp_eq_off[warp];
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int j0 = wlo; j0 < whi; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t u = j < whi ? key_at(j) : 0u;
+        const bool gt = j < whi && u > T, eq = j < whi && u == T;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const unsigned eq_rank = eq_run + __popc(eqm & lt_mask);
+        const bool sel = gt || (eq && eq_rank < need_eq);
+        const unsigned selm = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[pos + __popc(selm & lt_mask)] = j;
+        pos += __popc(selm);
+        eq_run += __popc(eqm);
+    }
+    cluster.sync();                        // the leader's shared memory outlives its readers
 }
 
 }  // namespace
@@ -127,9 +231,32 @@ cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score,
                           void* scratch, cudaStream_t st) {
     (void)p;
     (void)scratch;
-    select_topk_rows<<<s.batch * s.hkv, kSelectThreads, 0, st>>>(score, idx, s.seq_len, s.window,
-                                                                 s.budget);
-    return cudaGetLastError();
+    const int n = s.seq_len - s.window;
+    const int slice = (n + kCl - 1) / kCl;
+    const bool in_smem = slice <= kSliceCap;
+    const size_t dyn = in_smem ? (size_t)slice * sizeof(uint32_t) : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(s.batch * s.hkv * kCl);
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = dyn;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kCl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (in_smem) {
+        e = cudaFuncSetAttribute(select_cluster<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dyn);
+        if (e != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, select_cluster<true>, score, idx, s.seq_len, s.window,
+                                  s.budget, slice);
+    }
+    return cudaLaunchKernelEx(&cfg, select_cluster<false>, score, idx, s.seq_len, s.window,
+                              s.budget, slice);
 }
 
 }  // namespace kvp
