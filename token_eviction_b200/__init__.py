@@ -26,7 +26,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkvp.so")
+# KVP_LIBRARY may point at another build of the same library (e.g. one compiled with
+# device-side bounds checks); the default is the in-tree build.
+LIB_PATH = os.environ.get("KVP_LIBRARY", os.path.join(_HERE, "libkvp.so"))
 
 KVP_OK = 0
 STATUS_NAMES = {0: "KVP_OK", 1: "KVP_ERR_NULL", 2: "KVP_ERR_SHAPE", 3: "KVP_ERR_ALIGN",

@@ -37,24 +37,28 @@ def _stale() -> bool:
     return any(os.path.getmtime(f) > t for f in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, out: str | None = None,
+          defines: tuple = ()) -> str:
+    """Compile and link the library (to `out`, default in-tree; `defines` such as
+    "KVP_CHECKS" add -D flags, for a debug build with device-side bounds checks)."""
+    target = out or LIB
+    if not force and out is None and not defines and not _stale():
         return LIB
-    objdir = os.path.join(ROOT, "_build")
+    objdir = os.path.join(ROOT, "_build", "dbg" if defines else "rel")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [NVCC, *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
         objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = target + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

@@ -56,7 +56,7 @@ bool plan_of(const kvp_shape& s, Plan* p) {
     p->off_err = off;
     off += 256;
     p->off_part = off;
-    off += align_up((size_t)s.batch * s.hq * s.window * slots * sizeof(float2), 256);
+    off += align_up((size_t)s.batch * s.hq * s.window * p->maxslots * sizeof(float2), 256);
     p->off_select = off;
     off += 256;
     p->bytes = off;
@@ -121,6 +121,27 @@ extern "C" kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, con
         return KVP_ERR_CUDA;
     return KVP_OK;
 }
+
+#ifdef KVP_CHECKS
+// Debug builds only: copy out (and clear) the first failed device-side bounds check.
+extern "C" KVP_API int kvp_debug_take_check_unit(int unit, int* out4) {
+    int (*readers[3])(int*) = {take_check_score, take_check_select, take_check_compact};
+    if (unit < 0 || unit > 2) return -1;
+    return readers[unit](out4);
+}
+
+extern "C" KVP_API int kvp_debug_take_check(int* out4) {
+    int (*readers[3])(int*) = {take_check_score, take_check_select, take_check_compact};
+    out4[0] = out4[1] = out4[2] = out4[3] = 0;
+    for (auto rd : readers) {
+        int v[4];
+        if (rd(v) != 0) return -1;
+        if (v[0] != 0 && out4[0] == 0)
+            for (int i = 0; i < 4; ++i) out4[i] = v[i];
+    }
+    return 0;
+}
+#endif
 
 extern "C" const char* kvp_status_string(kvp_status status) {
     switch (status) {

@@ -17,7 +17,7 @@ __global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ k,
                                                    const int32_t* __restrict__ idx,
                                                    uint4* __restrict__ k_out,
                                                    uint4* __restrict__ v_out, int L, int B,
-                                                   int piece_shift, int total) {
+                                                   int piece_shift, int total, int rows_total) {
     const int stride = gridDim.x * blockDim.x;
     const int pmask = (1 << piece_shift) - 1;
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ k,
             a = __ldg(k + src);
             b = __ldg(v + src);
         }
+        if (!KVP_CHECK(row < rows_total, 301, row, rt)) continue;
         __stcs(k_out + e, a);
         __stcs(v_out + e, b);
     }
@@ -48,8 +49,13 @@ cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t
     const long long cap = (long long)sms * 8;  // 8 resident CTAs of 256 threads per SM
     const int grid = (int)(want < cap ? want : cap);
     gather_rows<<<grid, 256, 0, st>>>((const uint4*)k, (const uint4*)v, idx, (uint4*)k_out,
-                                      (uint4*)v_out, s.seq_len, s.budget, piece_shift, (int)total);
+                                      (uint4*)v_out, s.seq_len, s.budget, piece_shift, (int)total,
+                                      s.batch * s.hkv);
     return cudaGetLastError();
 }
+
+#ifdef KVP_CHECKS
+KVP_DEFINE_CHECK_READER(take_check_compact)
+#endif
 
 }  // namespace kvp

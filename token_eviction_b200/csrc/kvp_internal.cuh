@@ -59,4 +59,29 @@ cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t
 
 int num_sms();
 
+#ifdef KVP_CHECKS
+// Debug builds only: the first failed device-side bounds check (code, a, b) is recorded
+// here and the access skipped, instead of touching memory out of bounds.
+// One copy per translation unit (no relocatable device code); each unit exports a reader.
+static __device__ int g_kvp_check[4];
+#define KVP_DEFINE_CHECK_READER(fn)                                                        \
+    int fn(int* out4) {                                                                    \
+        if (cudaMemcpyFromSymbol(out4, g_kvp_check, 4 * sizeof(int)) != cudaSuccess) return -1; \
+        const int zero[4] = {0, 0, 0, 0};                                                  \
+        return cudaMemcpyToSymbol(g_kvp_check, zero, sizeof(zero)) == cudaSuccess ? 0 : -1; \
+    }
+int take_check_score(int* out4);
+int take_check_select(int* out4);
+int take_check_compact(int* out4);
+__device__ __forceinline__ void kvp_check_fail(int code, int a, int b) {
+    if (atomicCAS(&g_kvp_check[0], 0, code) == 0) {
+        g_kvp_check[1] = a;
+        g_kvp_check[2] = b;
+    }
+}
+#define KVP_CHECK(cond, code, a, b) ((cond) ? true : (kvp_check_fail((code), (a), (b)), false))
+#else
+#define KVP_CHECK(cond, code, a, b) true
+#endif
+
 }  // namespace kvp

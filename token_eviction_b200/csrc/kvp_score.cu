@@ -461,7 +461,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     const int r = m * kTile + lrow;
-                    if (m < p.mt && r < p.rows) {
+                    if (m < p.mt && r < p.rows && KVP_CHECK(slot >= 0 && slot < p.maxslots, 202, slot, head)) {
                         const bool mine = m >= mlo && m < mhi;
                         p.part[(size_t)(r0 + r) * p.maxslots + slot] =
                             mine ? make_float2(mrun[m], lrun[m]) : make_float2(-INFINITY, 0.f);
@@ -596,7 +596,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         __syncwarp();
                         if (lane == 0) ptx::mbar_arrive(&sb->combempty[cb]);
                     }
-                    if (j < p.L) {
+                    if (j < p.L && KVP_CHECK(head < p.total_tiles / p.tiles_per_head, 201, head, j)) {
                         const size_t o = (size_t)head * p.L + j;
                         p.score[o] = s1v * s2v;
                         if (p.s1) p.s1[o] = s1v;
@@ -785,5 +785,9 @@ cudaError_t launch_score(const kvp_shape& s, const Plan& plan, const uint16_t* q
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, qmap, kmap, vmap, p);
 }
+
+#ifdef KVP_CHECKS
+KVP_DEFINE_CHECK_READER(take_check_score)
+#endif
 
 }  // namespace kvp

@@ -218,7 +218,10 @@ select_cluster(const float* __restrict__ score, int32_t* __restrict__ idx, int L
         const unsigned eq_rank = eq_run + __popc(eqm & lt_mask);
         const bool sel = gt || (eq && eq_rank < need_eq);
         const unsigned selm = __ballot_sync(0xffffffffu, sel);
-        if (sel) out[pos + __popc(selm & lt_mask)] = j;
+        if (sel) {
+            const unsigned slot = pos + __popc(selm & lt_mask);
+            if (KVP_CHECK(slot < (unsigned)kk, 101, row, (int)slot)) out[slot] = j;
+        }
         pos += __popc(selm);
         eq_run += __popc(eqm);
     }
@@ -258,5 +261,9 @@ cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score,
     return cudaLaunchKernelEx(&cfg, select_cluster<false>, score, idx, s.seq_len, s.window,
                               s.budget, slice);
 }
+
+#ifdef KVP_CHECKS
+KVP_DEFINE_CHECK_READER(take_check_select)
+#endif
 
 }  // namespace kvp
