@@ -28,8 +28,9 @@
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls only enqueue
  *     work and never synchronise the host.
  *   - Argument errors are detected on the host before anything is launched; the outputs
- *     are then untouched. A launch failure returns KVP_ERR_CUDA (the CUDA error is
- *     consumed). Kernels contain no waits that can hang.
+ *     are then untouched. A launch failure returns KVP_ERR_CUDA; kvp_last_cuda_error()
+ *     names the CUDA error. Every device-side wait is bounded in time, so no kernel can
+ *     hang.
  */
 #ifndef KVP_H_
 #define KVP_H_
@@ -106,6 +107,10 @@ KVP_API kvp_status kvp_select(const kvp_shape* shape, const float* score, int32_
  */
 KVP_API kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
                                const int32_t* idx, uint16_t* k_out, uint16_t* v_out, void* stream);
+
+/* The name of the CUDA error behind the calling thread's most recent KVP_ERR_CUDA
+ * ("cudaSuccess" if there was none). Host-only; never fails. */
+KVP_API const char* kvp_last_cuda_error(void);
 
 /* A static, human-readable name of a status code. */
 KVP_API const char* kvp_status_string(kvp_status status);

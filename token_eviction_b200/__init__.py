@@ -49,13 +49,16 @@ class KvpShape(ctypes.Structure):
 class KvpError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {kvp_status_string(status)}")
+        msg = f"{what}: {kvp_status_string(status)}"
+        if status == 5:
+            msg += f" ({kvp_last_cuda_error()})"
+        super().__init__(msg)
 
 
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m token_eviction_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python token_eviction_b200/build.py` "
             "(there is no fallback implementation)")
     lib = ctypes.CDLL(LIB_PATH)
     P, S = ctypes.c_void_p, ctypes.POINTER(KvpShape)
@@ -69,6 +72,8 @@ def _load():
     lib.kvp_compact.restype = ctypes.c_int
     lib.kvp_status_string.argtypes = [ctypes.c_int]
     lib.kvp_status_string.restype = ctypes.c_char_p
+    lib.kvp_last_cuda_error.argtypes = []
+    lib.kvp_last_cuda_error.restype = ctypes.c_char_p
     return lib
 
 
@@ -79,7 +84,8 @@ _lib = _load()
 # enqueues one small memset of its workspace counters.
 KERNELS_PER_LAYER = 3
 
-EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact", "kvp_status_string")
+EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact", "kvp_status_string",
+            "kvp_last_cuda_error")
 
 
 def make_shape(batch, hq, hkv, head_dim, seq_len, window, budget) -> KvpShape:
@@ -97,6 +103,10 @@ def _as_shape(shape) -> KvpShape:
 
 def kvp_status_string(status: int) -> str:
     return _lib.kvp_status_string(int(status)).decode()
+
+
+def kvp_last_cuda_error() -> str:
+    return _lib.kvp_last_cuda_error().decode()
 
 
 def kvp_workspace_bytes(shape) -> int:

@@ -1,6 +1,8 @@
 """Build ``libkvp.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m token_eviction_b200.build [--force]
+    python token_eviction_b200/build.py [--force] [-v]
+
+(Run it as a script: importing the package loads the library this builds.)
 
 The library is plain C ABI over CUDA: every ``csrc/*.cu`` is compiled for
 ``sm_100a`` and linked into one shared object beside this file, with the CUDA runtime

@@ -69,6 +69,15 @@ using namespace kvp;
 
 static bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 
+// The CUDA error behind the calling thread's last KVP_ERR_CUDA (cudaSuccess if none).
+static thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+static kvp_status cuda_failed(cudaError_t e) {
+    t_last_cuda_error = e;
+    cudaGetLastError();  // clear the runtime's sticky copy of a launch error
+    return KVP_ERR_CUDA;
+}
+
 extern "C" size_t kvp_workspace_bytes(const kvp_shape* shape) {
     Plan p;
     if (!shape || !plan_of(*shape, &p)) return 0;
@@ -86,11 +95,9 @@ extern "C" kvp_status kvp_score(const kvp_shape* shape, const uint16_t* q_win, c
         return KVP_ERR_ALIGN;
     if (!workspace || workspace_bytes < p.bytes) return KVP_ERR_WORKSPACE;
     if (!aligned16(workspace)) return KVP_ERR_ALIGN;
-    if (launch_score(*shape, p, q_win, k, v, workspace, score, s1, s2, (cudaStream_t)stream) !=
-        cudaSuccess) {
-        cudaGetLastError();
-        return KVP_ERR_CUDA;
-    }
+    const cudaError_t e =
+        launch_score(*shape, p, q_win, k, v, workspace, score, s1, s2, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_failed(e);
     return KVP_OK;
 }
 
@@ -102,9 +109,9 @@ extern "C" kvp_status kvp_select(const kvp_shape* shape, const float* score, int
     if (!aligned16(score) || !aligned16(idx)) return KVP_ERR_ALIGN;
     if (!workspace || workspace_bytes < p.bytes) return KVP_ERR_WORKSPACE;
     if (!aligned16(workspace)) return KVP_ERR_ALIGN;
-    if (launch_select(*shape, p, score, idx, (char*)workspace + p.off_select,
-                      (cudaStream_t)stream) != cudaSuccess)
-        return KVP_ERR_CUDA;
+    const cudaError_t e =
+        launch_select(*shape, p, score, idx, (char*)workspace + p.off_select, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_failed(e);
     return KVP_OK;
 }
 
@@ -117,8 +124,8 @@ extern "C" kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, con
     if (!aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(k_out) ||
         !aligned16(v_out))
         return KVP_ERR_ALIGN;
-    if (launch_compact(*shape, k, v, idx, k_out, v_out, (cudaStream_t)stream) != cudaSuccess)
-        return KVP_ERR_CUDA;
+    const cudaError_t e = launch_compact(*shape, k, v, idx, k_out, v_out, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_failed(e);
     return KVP_OK;
 }
 
@@ -142,6 +149,16 @@ extern "C" KVP_API int kvp_debug_take_check(int* out4) {
     return 0;
 }
 #endif
+
+#ifdef KVP_TRACE
+namespace kvp { int take_trace(unsigned long long* out); }
+// Debug builds only: per-CTA %globaltimer stamps of the last scoring launch, [148][8].
+extern "C" KVP_API int kvp_debug_trace(unsigned long long* out) { return kvp::take_trace(out); }
+#endif
+
+extern "C" const char* kvp_last_cuda_error(void) {
+    return t_last_cuda_error == cudaSuccess ? "cudaSuccess" : cudaGetErrorName(t_last_cuda_error);
+}
 
 extern "C" const char* kvp_status_string(kvp_status status) {
     switch (status) {

@@ -34,8 +34,8 @@ struct Plan {
 // fewer, provided the workspace's slot count still covers every head.
 constexpr int kPlanGrid = 148;
 
-// Partial-softmax slots a CTA fills per KV head it touches (one per epilogue group).
-constexpr int kSlotsPerCta = 2;
+// Partial-softmax slots a CTA fills per KV head it touches.
+constexpr int kSlotsPerCta = 1;
 
 bool plan_of(const kvp_shape& s, Plan* p);
 

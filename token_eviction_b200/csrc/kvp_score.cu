@@ -53,27 +53,46 @@ constexpr int kEpiThreads = 128 * kEpiGroups;
 constexpr int kThreads = 64 + kEpiThreads;        // + TMA warp + MMA warp
 constexpr int kMaxStages = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kStageCols = 256;              // one accumulator stage per group
+constexpr uint32_t kMaxStageCols = 256;           // widest accumulator stage
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s on any single wait
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMinSmem = 116 * 1024;              // forces one CTA per SM (TMEM is taken whole)
 constexpr int kQBoxRows = 64;
+constexpr size_t kBarBytes = 512;                 // shared memory reserved for SmemBars
+
+#ifdef KVP_TRACE
+// Debug builds only: %globaltimer stamps per CTA at phase boundaries.
+__device__ unsigned long long g_kvp_trace[kPlanGrid][8];
+#define KVP_STAMP(i) (g_kvp_trace[blockIdx.x][(i)] = ptx::globaltimer_ns())
+// per-tile events of the first 4 CTAs: [cta][tile][event]
+__device__ unsigned long long g_kvp_ttrace[4][64][8];
+// MMA-thread steps of the first 4 CTAs (clock64): [cta][tile][step]
+__device__ long long g_kvp_mtrace[4][64][12];
+#define KVP_MSTAMP(t, e) ((blockIdx.x < 4 && (t) < 64) ? (void)(g_kvp_mtrace[blockIdx.x][(t)][(e)] = clock64()) : (void)0)
+#define KVP_TSTAMP(t, e) \
+    ((blockIdx.x < 4 && (t) < 64) ? (void)(g_kvp_ttrace[blockIdx.x][(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
+#else
+#define KVP_STAMP(i) ((void)0)
+#define KVP_TSTAMP(t, e) ((void)0)
+#define KVP_MSTAMP(t, e) ((void)0)
+#endif
 
 // error codes recorded in the workspace (first one wins)
 enum : int { kErrWaitTma = 1, kErrWaitMma = 2, kErrWaitEpi = 3, kErrWaitPeers = 4 };
 
 struct Params {
     int L, w, G, rows, hq, hkv, D;
-    int mt;              // 128-row tiles covering the query group (phase 0 M tiles)
-    int mt0;             // split mode: M tiles in stage 0 (the rest in stage 1)
     int qrows;           // query rows staged in shared memory (rows rounded up to 64)
     int n1, n2;          // phase 1 MMA N of the two column chunks (n2 = 0: one chunk)
     int split;           // 0: groups alternate tiles; 1: every tile split over both stages
+    int stage_cols;      // TMEM columns per accumulator stage (128 or 256)
+    int spg;             // accumulator stages per epilogue group (2 when a stage is 128 wide)
     int tiles_per_head, total_tiles, grid, maxslots;
     int nk, nv;          // K and V ring depths
     float scale2;        // log2(e) / sqrt(d)
     uint32_t q_bytes, k_bytes, v_bytes;
-    uint32_t off_q, off_k, off_v, off_lse, off_bar;
+    uint32_t off_q, off_k, off_v, off_lse, off_cw, off_bar;
+    int cw_stride;       // floats per epilogue warp of phase 0 row offsets
     float* score;
     float* s1;
     float* s2;
@@ -85,7 +104,7 @@ struct Params {
 struct SmemBars {
     uint64_t kfull[kMaxStages], kempty[kMaxStages];
     uint64_t vfull[kMaxStages], vempty[kMaxStages];
-    uint64_t accfull[2], accempty[2];
+    uint64_t accfull[4], accempty[4];
     uint64_t combfull[2], combempty[2];
     uint64_t qfull, qempty, fin;
     uint64_t epi;        // rendezvous of all epilogue threads
@@ -128,6 +147,19 @@ __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
     return *reinterpret_cast<uint32_t*>(&m);
 }
 
+// Accumulator stage that epilogue group g uses for the CTA's tile number i, and the
+// parity of that use. Alternate-tile mode: group i & 1 takes tile i, cycling through its
+// spg stages (stages g, g + 2); split mode: group g takes stage g of every tile.
+__device__ __forceinline__ int acc_stage(int split, int spg, int i, int g, uint32_t& parity) {
+    if (split) {
+        parity = (uint32_t)i & 1u;
+        return g;
+    }
+    const int u = i >> 1;
+    parity = (uint32_t)(u / spg) & 1u;
+    return g + 2 * (u % spg);
+}
+
 // Segments of a CTA's run: maximal stretches of tiles within one KV head.
 struct RunIter {
     long long t, end;
@@ -143,39 +175,60 @@ struct RunIter {
     }
 };
 
-__device__ __forceinline__ float tree_max32(const float (&v)[32]) {
-    float m[16];
+// Butterfly reduce-scatter across the 32 lanes of a warp: v[i] holds this lane's value of
+// column i; on return lane L's v[0] holds the maximum (kMax) or sum over all 32 lanes of
+// column L. Five rounds, 31 shuffles.
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32]) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) m[e] = fmaxf(v[e], v[e + 16]);
+    for (int k = 16; k >= 1; k >>= 1) {
+        const bool upper = (lane & k) != 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], m[e + 8]);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) m[e] = fmaxf(m[e], m[e + 4]);
-    return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
+        for (int i = 0; i < k; ++i) {
+            const float send = upper ? v[i] : v[i + k];
+            const float keep = upper ? v[i + k] : v[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, k);
+            v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+    return v[0];
 }
 
-// Phase 0, one 32-key chunk of one query row: fold the chunk into the running (m, l).
-// `last` is the last key position the row sees; `key0` the chunk's first key.
-__device__ __forceinline__ void lse_chunk(float (&v)[32], bool full, int key0, int last,
-                                          float scale2, float& mrun, float& lrun) {
-    if (!full) {
+// Phase 0, one 32-column chunk for one key per thread: v[i] is the key's raw logit
+// against query row (chunk column) i, masked to -inf where not visible. cw[0..31] are the
+// warp's running offsets of those rows (log2 units, shared memory). Returns, in lane L,
+// the warp's sum over its 32 keys of 2^(t - cw) for column L; on overflow (a logit far
+// above its row's offset) the offsets of the chunk are raised first and *lsum (lane L's
+// running sum of column L) rescaled to match.
+__device__ __forceinline__ float lse_chunk_t(const float (&v)[32], float* cw, float scale2,
+                                             float& lsum) {
+    const int lane = threadIdx.x & 31;
+    float e[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-            if (key0 + e > last) v[e] = -INFINITY;
+    for (int i = 0; i < 32; i += 4) {
+        const float4 c4 = *(const float4*)(cw + i);
+        e[i + 0] = ptx::ex2(fmaf(v[i + 0], scale2, -c4.x));
+        e[i + 1] = ptx::ex2(fmaf(v[i + 1], scale2, -c4.y));
+        e[i + 2] = ptx::ex2(fmaf(v[i + 2], scale2, -c4.z));
+        e[i + 3] = ptx::ex2(fmaf(v[i + 3], scale2, -c4.w));
     }
-    const float cm = tree_max32(v);
-    if (cm == -INFINITY) return;
-    const float mn = fmaxf(mrun, cm * scale2);
-    float a0 = lrun * ptx::ex2(mrun - mn), a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    float sum = warp_reduce_scatter32<false>(e);
+    if (__any_sync(0xffffffffu, !(sum < INFINITY))) {
+        // rare: raise each column's offset to the column's maximum where that is higher
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-        a0 += ptx::ex2(fmaf(v[e + 0], scale2, -mn));
-        a1 += ptx::ex2(fmaf(v[e + 1], scale2, -mn));
-        a2 += ptx::ex2(fmaf(v[e + 2], scale2, -mn));
-        a3 += ptx::ex2(fmaf(v[e + 3], scale2, -mn));
+        for (int i = 0; i < 32; ++i) e[i] = fmaf(v[i], scale2, -cw[i]);
+        float d = warp_reduce_scatter32<true>(e);
+        d = d > 0.f ? d : 0.f;                    // also maps NaN (all masked) to 0
+        lsum *= ptx::ex2(-d);
+        __syncwarp();
+        cw[lane] += d;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) e[i] = ptx::ex2(fmaf(v[i], scale2, -cw[i]));
+        sum = warp_reduce_scatter32<false>(e);
     }
-    lrun = (a0 + a1) + (a2 + a3);
-    mrun = mn;
+    return sum;
 }
 
 // Phase 1, one 32-column chunk of one key: add 2^(t - lse2[n]) over the chunk's valid
@@ -216,8 +269,11 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     uint8_t* Qs = smem + p.off_q;
     uint8_t* Ks = smem + p.off_k;
     uint8_t* Vs = smem + p.off_v;
-    float* lse2 = (float*)(smem + p.off_lse);          // [512]
-    float* comb = lse2 + kMaxGroupRows;                 // [2][128] partial S1 handoff
+    float* lse2 = (float*)(smem + p.off_lse);          // [rows, padded to 4]
+    float* comb = lse2 + ((p.rows + 3) & ~3);           // [2][128] partial S1 handoff (split mode)
+    // phase 0: [8 warps][cw_stride] row offsets; at the end of a head the same bytes stage
+    // the warps' (offset, sum) pairs as float2 [8][cw_stride]
+    float* cw_all = (float*)(smem + p.off_cw);
     SmemBars* sb = (SmemBars*)(smem + p.off_bar);
 
     constexpr int kHalves = D / 64;                 // 128-byte swizzle rows per operand row
@@ -236,9 +292,11 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             ptx::mbar_init(&sb->vfull[s], 1);
             ptx::mbar_init(&sb->vempty[s], 4);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < 4; ++s) {
             ptx::mbar_init(&sb->accfull[s], 1);
             ptx::mbar_init(&sb->accempty[s], 4);
+        }
+        for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&sb->combfull[s], 4);
             ptx::mbar_init(&sb->combempty[s], 4);
         }
@@ -262,6 +320,13 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sb->tmem_base;
+    if (threadIdx.x == 0) KVP_STAMP(0);
+#ifdef KVP_TRACE
+    if (threadIdx.x == 0 && blockIdx.x < 4) {
+        g_kvp_ttrace[blockIdx.x][63][0] = clock64();
+        g_kvp_ttrace[blockIdx.x][63][1] = ptx::globaltimer_ns();
+    }
+#endif
 
     auto group_row0 = [&](int bh) {
         const int b = bh / p.hkv, h = bh % p.hkv;
@@ -295,6 +360,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
                         const int s = kit % p.nk;
                         if (!(ok = wait_phase(&sb->kempty[s], ((kit / p.nk) & 1) ^ 1, sb, p.err, kErrWaitTma))) break;
+                        KVP_TSTAMP(kit, 0);
                         ptx::mbar_arrive_expect_tx(&sb->kfull[s], p.k_bytes);
                         for (int c = 0; c < kHalves; ++c)
                             ptx::tma_load_3d(Ks + s * kstage + c * kHalfTile, &kmap, &sb->kfull[s],
@@ -303,6 +369,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         if (phase == 1) {
                             const int sv = vit % p.nv;
                             if (!(ok = wait_phase(&sb->vempty[sv], ((vit / p.nv) & 1) ^ 1, sb, p.err, kErrWaitTma))) break;
+                            KVP_TSTAMP(kit - 1, 6);
                             ptx::mbar_arrive_expect_tx(&sb->vfull[sv], p.v_bytes);
                             ptx::tma_load_3d(Vs + sv * vstage, &vmap, &sb->vfull[sv], 0, key0, head,
                                              pol_stream);
@@ -310,6 +377,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         }
                     }
                 }
+                KVP_STAMP(1 + phase);
             }
             // Never leave with copies in flight: wait for the last load of every stage.
             for (int i = max(0, kit - p.nk); i < kit; ++i)
@@ -321,7 +389,6 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc0 = ptx::idesc_bf16_f32(128, kTile);
             const uint32_t idesc1a = ptx::idesc_bf16_f32(128, p.n1);
             const uint32_t idesc1b = ptx::idesc_bf16_f32(128, p.n2 > 0 ? p.n2 : 16);
             const uint32_t q_addr = ptx::smem_u32(Qs), k_addr = ptx::smem_u32(Ks);
@@ -341,40 +408,46 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     for (long long t = a; t < b; ++t) {
                         const int s = kit % p.nk;
                         if (!(ok = wait_phase(&sb->kfull[s], (kit / p.nk) & 1, sb, p.err, kErrWaitMma))) break;
+                        KVP_TSTAMP(kit, 1);
+                        KVP_MSTAMP(kit, 0);
                         const uint32_t kbase = k_addr + s * kstage;
                         // stages written for this tile: one (alternating) or both (split)
-                        const int st_lo = p.split ? 0 : (ait & 1);
-                        const int st_hi = p.split ? 1 : (ait & 1);
-                        const uint32_t use_parity = p.split ? (ait & 1) : ((ait >> 1) & 1);
-                        for (int st = st_lo; st <= st_hi && ok; ++st) {
+                        const int g_lo = p.split ? 0 : (ait & 1);
+                        const int g_hi = p.split ? 1 : (ait & 1);
+                        for (int g = g_lo; g <= g_hi && ok; ++g) {
+                            uint32_t use_parity;
+                            const int st = acc_stage(p.split, p.spg, ait, g, use_parity);
                             if (!(ok = wait_phase(&sb->accempty[st], use_parity ^ 1, sb, p.err, kErrWaitMma))) break;
+                            KVP_TSTAMP(kit, 2);
+                            KVP_MSTAMP(kit, 1);
                             ptx::tc_fence_after();
-                            const uint32_t d0 = tmem + (uint32_t)st * kStageCols;
+                            KVP_MSTAMP(kit, 2);
+                            const uint32_t d0 = tmem + (uint32_t)(st * p.stage_cols);
+                            // descriptors of the first k-step; later k-steps add byte
+                            // offsets (in 16-byte units) to the start-address field
+                            const uint64_t kdesc0 = ptx::sw128_kmajor_desc(kbase);
+                            const uint64_t qdesc0 = ptx::sw128_kmajor_desc(q_addr);
+                            const bool first_chunk = !p.split || g == 0;
+                            const bool second_chunk = p.n2 > 0 && (!p.split || g == 1);
+                            const uint32_t n2_col = p.split ? 0u : (uint32_t)p.n1;
+#pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
-                                const int c = ks >> 2, kk = ks & 3;
-                                const uint32_t koff = kbase + c * kHalfTile + kk * 32;
-                                const uint32_t qoff = q_addr + c * qhalf + kk * 32;
-                                if (phase == 0) {
-                                    const int mlo = p.split ? st * p.mt0 : 0;
-                                    const int mhi = p.split ? (st ? p.mt : p.mt0) : p.mt;
-                                    for (int m = mlo; m < mhi; ++m)
-                                        ptx::mma_bf16_ss(d0 + (m - mlo) * kTile,
-                                                         ptx::sw128_kmajor_desc(qoff + m * kHalfTile),
-                                                         ptx::sw128_kmajor_desc(koff), idesc0, ks > 0);
-                                } else {
-                                    const uint64_t adesc = ptx::sw128_kmajor_desc(koff);
-                                    if (!p.split || st == 0)
-                                        ptx::mma_bf16_ss(d0, adesc, ptx::sw128_kmajor_desc(qoff), idesc1a, ks > 0);
-                                    if (p.n2 > 0 && (!p.split || st == 1))
-                                        ptx::mma_bf16_ss(d0 + (p.split ? 0 : p.n1), adesc,
-                                                         ptx::sw128_kmajor_desc(qoff + p.n1 * 128),
-                                                         idesc1b, ks > 0);
-                                }
+                                const uint32_t koff = (uint32_t)((ks >> 2) * kHalfTile + (ks & 3) * 32) >> 4;
+                                const uint32_t qoff = ((ks >> 2) * qhalf + (ks & 3) * 32) >> 4;
+                                const uint64_t kd = kdesc0 + koff;
+                                if (first_chunk)
+                                    ptx::mma_bf16_ss(d0, kd, qdesc0 + qoff, idesc1a, ks > 0);
+                                if (second_chunk)
+                                    ptx::mma_bf16_ss(d0 + n2_col, kd, qdesc0 + qoff + (uint32_t)(p.n1 * 128 >> 4),
+                                                     idesc1b, ks > 0);
+                                KVP_MSTAMP(kit, 3 + (ks & 7));
                             }
                             ptx::mma_commit(&sb->accfull[st]);
                         }
                         if (!ok) break;
                         ptx::mma_commit(&sb->kempty[s]);
+                        KVP_TSTAMP(kit, 3);
+                        KVP_MSTAMP(kit, 11);
                         ++kit;
                         ++ait;
                     }
@@ -392,6 +465,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         if (more && nh != cur) ptx::mma_commit(&sb->qempty);
                     }
                 }
+                KVP_STAMP(3 + phase);
             }
             // all MMAs issued by this thread have completed before TMEM is released
             ptx::mma_commit(&sb->fin);
@@ -403,69 +477,134 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const int wg = et >> 7;                           // epilogue group = TMEM stage
         const int quarter = warp & 3;                     // TMEM lane quarter of this warp
         const int lrow = quarter * 32 + lane;             // lane: query row (phase 0) / key (phase 1)
-        const uint32_t tstage = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)wg * kStageCols;
+        const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);   // this warp's lanes
         const int window0 = p.L - p.w;                    // first window position
-        const int mlo = p.split ? wg * p.mt0 : 0;         // phase 0 M tiles of this group
-        const int mhi = p.split ? (wg ? p.mt : p.mt0) : p.mt;
+        // columns (query rows) this group's TMEM stage holds: all rows when the groups
+        // alternate tiles, one half each when every tile is split across both stages
+        const int col0 = (p.split && wg == 1) ? p.n1 : 0;
+        const int ncols = p.split ? (wg == 0 ? p.n1 : p.rows - p.n1) : p.rows;
+        const int nch = (ncols + 31) >> 5;
+        const int warp8 = et >> 5;                        // epilogue warp 0..7
+        float* cwp = cw_all + warp8 * p.cw_stride;        // this warp's row offsets
         int ait = 0;
         uint32_t epi_phase = 0;
         bool ok = true;
-        // ---- phase 0: per-row running max and sum over this CTA's keys of each head
+        // ---- phase 0: per query row, each warp's running offset and sum of 2^(t - offset)
+        //      over its keys (thread = key, TMEM columns = query rows)
         {
             RunIter it(t0, t1, p.tiles_per_head);
             int head;
             long long a, b;
             while (ok && it.next(head, a, b)) {
-                float mrun[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                float lrun[4] = {0.f, 0.f, 0.f, 0.f};
+                float lw[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                bool first_tile = true;
                 for (long long t = a; t < b && ok; ++t, ++ait) {
                     if (!p.split && (ait & 1) != wg) continue;       // the other group's tile
-                    const uint32_t parity = p.split ? (ait & 1) : ((ait >> 1) & 1);
-                    if (!(ok = wait_phase(&sb->accfull[wg], parity, sb, p.err, kErrWaitEpi))) break;
+                    uint32_t parity;
+                    const int st = acc_stage(p.split, p.spg, ait, wg, parity);
+                    const uint32_t tstage = tlane + (uint32_t)(st * p.stage_cols);
+                    if (!(ok = wait_phase(&sb->accfull[st], parity, sb, p.err, kErrWaitEpi))) break;
+                    if (lrow == 0) KVP_TSTAMP(ait, 4);
                     ptx::tc_fence_after();
                     const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
-                    const bool full = key0 + kTile - 1 <= window0;   // every row sees every key
+                    const int j = key0 + lrow;                       // this thread's key
+                    const bool full = key0 + kTile - 1 <= window0;
+                    const int jw = j - window0;                      // > 0 only inside the window
+                    // one 32-column chunk: mask, (first tile) set offsets, fold into lw
+                    auto chunk0 = [&](float (&v)[32], int c) {
+                        if (!full || (c + 1) * 32 > ncols) {
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        if (m < mlo || m >= mhi) continue;           // uniform across the group
-                        const int r = m * kTile + lrow;
-                        const int last = window0 + (r % p.w);        // last key row r sees
-                        const uint32_t tb = tstage + (uint32_t)(m - mlo) * kTile;
-                        float x[32], y[32];
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tb, x);
-                        ptx::tmem_ld_wait(x);
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tb + 32, y);
-                        lse_chunk(x, full, key0, last, p.scale2, mrun[m], lrun[m]);
-                        ptx::tmem_ld_wait(y);
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tb + 64, x);
-                        lse_chunk(y, full, key0 + 32, last, p.scale2, mrun[m], lrun[m]);
-                        ptx::tmem_ld_wait(x);
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tb + 96, y);
-                        lse_chunk(x, full, key0 + 64, last, p.scale2, mrun[m], lrun[m]);
-                        ptx::tmem_ld_wait(y);
-                        lse_chunk(y, full, key0 + 96, last, p.scale2, mrun[m], lrun[m]);
+                            for (int e = 0; e < 32; ++e) {
+                                const int n = c * 32 + e;
+                                if (n >= ncols || jw > (col0 + n) % p.w) v[e] = -INFINITY;
+                            }
+                        }
+                        if (first_tile) {
+                            // offsets from this (first) tile: each row's maximum over the warp's keys
+                            float m[32];
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) m[e] = v[e];
+                            const float cmax = warp_reduce_scatter32<true>(m);
+                            __syncwarp();
+                            cwp[c * 32 + lane] = cmax == -INFINITY ? -1e30f : cmax * p.scale2;
+                            __syncwarp();
+                        }
+                        float lcur = 0.f;              // lane L: running sum of column c*32+L
+#pragma unroll
+                        for (int cc = 0; cc < 8; ++cc)
+                            if (cc == c) lcur = lw[cc];
+                        lcur += lse_chunk_t(v, cwp + c * 32, p.scale2, lcur);
+#pragma unroll
+                        for (int cc = 0; cc < 8; ++cc)
+                            if (cc == c) lw[cc] = lcur;
+                    };
+                    float x[32], y[32];
+                    __syncwarp();
+                    ptx::tmem_ld_32x32b_x32(tstage, x);
+                    ptx::tmem_ld_wait(x);
+                    for (int c = 0; c < nch; c += 2) {
+                        const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
+                        if (has1) {
+                            __syncwarp();
+                            ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
+                        }
+                        chunk0(x, c);
+                        if (has1) {
+                            ptx::tmem_ld_wait(y);
+                            if (has2) {
+                                __syncwarp();
+                                ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
+                            }
+                            chunk0(y, c + 1);
+                            if (has2) ptx::tmem_ld_wait(x);
+                        }
                     }
+                    first_tile = false;
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[wg]);
+                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[st]);
+                    if (lrow == 0) KVP_TSTAMP(ait, 5);
                 }
                 if (!ok) break;
-                // publish this group's partials for `head` into its own slot
-                const long long first = (long long)head * p.tiles_per_head;
-                const int slot = ((int)blockIdx.x - owner_of(first, T, p.grid)) * kSlotsPerCta + wg;
-                const int r0 = group_row0(head);
+                // Combine the warps' (offset, sum) of every row inside the CTA, then publish
+                // one slot per row. The staging buffer aliases the offsets, so each lane
+                // first takes its own offsets into registers.
+                float cwr[8];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int r = m * kTile + lrow;
-                    if (m < p.mt && r < p.rows && KVP_CHECK(slot >= 0 && slot < p.maxslots, 202, slot, head)) {
-                        const bool mine = m >= mlo && m < mhi;
-                        p.part[(size_t)(r0 + r) * p.maxslots + slot] =
-                            mine ? make_float2(mrun[m], lrun[m]) : make_float2(-INFINITY, 0.f);
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int n = cc * 32 + lane;
+                    cwr[cc] = (n < ncols) ? cwp[n] : 0.f;
+                }
+                if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
+                float2* stage = reinterpret_cast<float2*>(cw_all) + warp8 * p.cw_stride;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int n = cc * 32 + lane;
+                    if (n < ncols)
+                        stage[n] = first_tile ? make_float2(-INFINITY, 0.f) : make_float2(cwr[cc], lw[cc]);
+                }
+                if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
+                const long long first = (long long)head * p.tiles_per_head;
+                const int slot = (int)blockIdx.x - owner_of(first, T, p.grid);
+                const int r0 = group_row0(head);
+                for (int r = et; r < p.rows; r += kEpiThreads) {
+                    // warps holding row r: all eight, or the four of the group owning it
+                    const int g = (p.split && r >= p.n1) ? 1 : 0;
+                    const int n = r - (g ? p.n1 : 0);
+                    const int w_lo = p.split ? 4 * g : 0, w_hi = p.split ? 4 * g + 4 : 8;
+                    float M = -INFINITY, S = 0.f;
+                    for (int w = w_lo; w < w_hi; ++w) {
+                        const float2 ml = reinterpret_cast<const float2*>(cw_all)[w * p.cw_stride + n];
+                        if (ml.y == 0.f) continue;
+                        if (ml.x > M) {
+                            S = S * ptx::ex2(M - ml.x) + ml.y;
+                            M = ml.x;
+                        } else {
+                            S += ml.y * ptx::ex2(ml.x - M);
+                        }
                     }
+                    if (KVP_CHECK(slot >= 0 && slot < p.maxslots, 202, slot, head))
+                        p.part[(size_t)(r0 + r) * p.maxslots + slot] = make_float2(M, S);
                 }
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
                 if (et == 0) {
@@ -474,8 +613,10 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 }
             }
         }
+        if (et == 0) KVP_STAMP(5);
         // ---- phase 1: scores
         {
+            bool first_seg = true;
             RunIter it(t0, t1, p.tiles_per_head);
             int head;
             long long a, b;
@@ -498,22 +639,39 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     }
                 }
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
+                if (et == 0 && first_seg) KVP_STAMP(6);
+                first_seg = false;
                 if (*(volatile int*)&sb->abort_flag) {
                     ok = false;
                     break;
                 }
                 const int r0 = group_row0(head);
                 const int nslots = touch * kSlotsPerCta;
-                for (int r = et; r < p.rows; r += kEpiThreads) {
-                    const float2* pr = p.part + (size_t)(r0 + r) * p.maxslots;
-                    float M = -INFINITY;
-                    for (int s = 0; s < nslots; ++s) M = fmaxf(M, __ldcg(&pr[s].x));
-                    float sum = 0.f;
-                    for (int s = 0; s < nslots; ++s) {
-                        const float2 ml = __ldcg(pr + s);
-                        if (ml.x != -INFINITY) sum += ml.y * ptx::ex2(ml.x - M);
+                // Two threads per row, each folding every other slot with independent
+                // loads (online max/sum), then one exchange with the partner lane.
+                for (int base = 0; base < 2 * p.rows; base += kEpiThreads) {
+                    const int r2 = base + et, r = r2 >> 1;
+                    float M = -INFINITY, S = 0.f;
+                    if (r < p.rows) {
+                        const float2* pr = p.part + (size_t)(r0 + r) * p.maxslots;
+#pragma unroll 4
+                        for (int sl = r2 & 1; sl < nslots; sl += 2) {
+                            const float2 ml = __ldcg(pr + sl);
+                            if (ml.x == -INFINITY || ml.y == 0.f) continue;
+                            if (ml.x > M) {
+                                S = S * ptx::ex2(M - ml.x) + ml.y;
+                                M = ml.x;
+                            } else {
+                                S += ml.y * ptx::ex2(ml.x - M);
+                            }
+                        }
                     }
-                    lse2[r] = M + __log2f(sum);
+                    const float Mo = __shfl_xor_sync(0xffffffffu, M, 1);
+                    const float So = __shfl_xor_sync(0xffffffffu, S, 1);
+                    const float Mt = fmaxf(M, Mo);
+                    const float St = (M == -INFINITY ? 0.f : S * ptx::ex2(M - Mt)) +
+                                     (Mo == -INFINITY ? 0.f : So * ptx::ex2(Mo - Mt));
+                    if (r < p.rows && (r2 & 1) == 0) lse2[r] = Mt + __log2f(St);
                 }
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
                 for (long long t = a; t < b && ok; ++t, ++ait, ++pt) {
@@ -528,6 +686,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         // rotated order per lane (conflict-free shared-memory reads)
                         const int sv = pt % p.nv;
                         if (!(ok = wait_phase(&sb->vfull[sv], (pt / p.nv) & 1, sb, p.err, kErrWaitEpi))) break;
+                        if (lrow == 0) KVP_TSTAMP(ait, 7);
                         const uint4* vrow = (const uint4*)(Vs + sv * vstage + lrow * (D * 2));
                         constexpr int kPieces = D * 2 / 16;
                         uint32_t mx = 0;
@@ -544,8 +703,11 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         if (lane == 0) ptx::mbar_arrive(&sb->vempty[sv]);
                     }
                     // S1 over this group's columns
-                    const uint32_t parity = p.split ? (ait & 1) : ((ait >> 1) & 1);
-                    if (!(ok = wait_phase(&sb->accfull[wg], parity, sb, p.err, kErrWaitEpi))) break;
+                    uint32_t parity;
+                    const int st = acc_stage(p.split, p.spg, ait, wg, parity);
+                    const uint32_t tstage = tlane + (uint32_t)(st * p.stage_cols);
+                    if (!(ok = wait_phase(&sb->accfull[st], parity, sb, p.err, kErrWaitEpi))) break;
+                    if (lrow == 0) KVP_TSTAMP(ait, 4);
                     ptx::tc_fence_after();
                     const bool full = key0 + kTile - 1 <= window0;
                     const int jw = j - window0;                     // > 0 only inside the window
@@ -578,7 +740,8 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     }
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[wg]);
+                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[st]);
+                    if (lrow == 0) KVP_TSTAMP(ait, 5);
                     float s1v = (a0 + a1) + (a2 + a3);
                     if (p.split) {
                         // hand the second group's partial to the first
@@ -607,6 +770,13 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         }
     }
 
+    if (threadIdx.x == 64) KVP_STAMP(7);
+#ifdef KVP_TRACE
+    if (threadIdx.x == 64 && blockIdx.x < 4) {
+        g_kvp_ttrace[blockIdx.x][63][2] = clock64();
+        g_kvp_ttrace[blockIdx.x][63][3] = ptx::globaltimer_ns();
+    }
+#endif
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -665,7 +835,6 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.hq = s.hq;
     p.hkv = s.hkv;
     p.D = D;
-    p.mt = (plan.rows + kTile - 1) / kTile;
     const int npad = (plan.rows + 15) / 16 * 16;
     if (npad <= 256) {
         p.n1 = npad;
@@ -674,8 +843,10 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
         p.n1 = (npad / 2 + 15) / 16 * 16;
         p.n2 = npad - p.n1;
     }
-    p.split = plan.rows > (int)kStageCols ? 1 : 0;
-    p.mt0 = (p.mt + 1) / 2;
+    p.split = plan.rows > (int)kMaxStageCols ? 1 : 0;
+    // two 128-column stages per group when a tile's accumulator fits 128 columns
+    p.stage_cols = (!p.split && (plan.rows + 31) / 32 * 32 <= 128) ? 128 : 256;
+    p.spg = p.stage_cols == 128 ? 2 : 1;
     p.tiles_per_head = plan.tiles_per_head;
     p.total_tiles = plan.total_tiles;
     p.grid = std::min(plan.grid, sms);
@@ -698,14 +869,25 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.q_bytes = qbytes;
     p.k_bytes = tile_bytes;
     p.v_bytes = tile_bytes;
-    // shared memory: Q | K ring | V ring | lse2 + handoff | barriers (+1 KB to align the base)
+    // shared memory: Q | K ring | V ring | lse2 + handoff | phase 0 row offsets | barriers
+    // (+1 KB to align the base)
+    const int group_cols = p.split ? std::max(p.n1, plan.rows - p.n1) : plan.rows;
+    p.cw_stride = (group_cols + 31) / 32 * 32;
+    const size_t cw_bytes = (size_t)(kEpiThreads / 32) * p.cw_stride * sizeof(float2);
+    // Alternate-tile mode: both epilogue groups read V stages, each its own tiles; with an
+    // even V ring a group only ever waits on its own stages, one phase ahead at most (an
+    // odd ring would make a group wait two phases ahead on a shared stage, where the
+    // parity test cannot tell the phases apart). Split mode: group 0 alone reads V.
     const int choices[5][2] = {{4, 2}, {3, 2}, {2, 2}, {3, 1}, {2, 1}};
-    const size_t lse_bytes = (kMaxGroupRows + 2 * kTile) * sizeof(float);
-    const size_t fixed = lse_bytes + 256 + 1024;
+    // lse2[rows] (16-byte padded), then the split-mode handoff comb[2][128]
+    const size_t lse_floats = (size_t)((plan.rows + 3) / 4 * 4);
+    const size_t lse_bytes = (lse_floats + (p.split ? 2 * kTile : 0)) * sizeof(float);
+    const size_t fixed = lse_bytes + cw_bytes + kBarBytes + 1024;
     size_t total = 0;
     bool fit = false;
     for (auto& c : choices) {
         total = qbytes + (size_t)(c[0] + c[1]) * tile_bytes + fixed;
+        if (!p.split && c[1] % 2 != 0) continue;
         if (total <= (size_t)kSmemLimit) {
             p.nk = c[0];
             p.nv = c[1];
@@ -718,8 +900,9 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.off_k = qbytes;
     p.off_v = p.off_k + p.nk * tile_bytes;
     p.off_lse = p.off_v + p.nv * tile_bytes;
-    p.off_bar = p.off_lse + (uint32_t)lse_bytes;
-    static_assert(sizeof(SmemBars) <= 256, "barrier block");
+    p.off_cw = p.off_lse + (uint32_t)lse_bytes;
+    p.off_bar = p.off_cw + (uint32_t)cw_bytes;
+    static_assert(sizeof(SmemBars) <= kBarBytes, "barrier block");
     L->grid = p.grid;
     L->smem = std::max(total, (size_t)kMinSmem);
     return true;
@@ -788,6 +971,13 @@ cudaError_t launch_score(const kvp_shape& s, const Plan& plan, const uint16_t* q
 
 #ifdef KVP_CHECKS
 KVP_DEFINE_CHECK_READER(take_check_score)
+#endif
+#ifdef KVP_TRACE
+int take_trace(unsigned long long* out) {
+    if (cudaMemcpyFromSymbol(out, g_kvp_trace, sizeof(g_kvp_trace)) != cudaSuccess) return -1;
+    if (cudaMemcpyFromSymbol(out + 148 * 8, g_kvp_ttrace, sizeof(g_kvp_ttrace)) != cudaSuccess) return -1;
+    return cudaMemcpyFromSymbol(out + 148 * 8 + 4 * 64 * 8, g_kvp_mtrace, sizeof(g_kvp_mtrace)) == cudaSuccess ? 0 : -1;
+}
 #endif
 
 }  // namespace kvp
