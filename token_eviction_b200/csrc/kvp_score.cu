@@ -69,8 +69,11 @@ __device__ unsigned long long g_kvp_ttrace[4][64][8];
 // MMA-thread steps of the first 4 CTAs (clock64): [cta][tile][step]
 __device__ long long g_kvp_mtrace[4][64][12];
 #define KVP_MSTAMP(t, e) ((blockIdx.x < 4 && (t) < 64) ? (void)(g_kvp_mtrace[blockIdx.x][(t)][(e)] = clock64()) : (void)0)
+__device__ __forceinline__ int kvp_trace_slot() {
+    return blockIdx.x == 0 ? 0 : blockIdx.x == 18 ? 1 : blockIdx.x == 73 ? 2 : blockIdx.x == 147 ? 3 : -1;
+}
 #define KVP_TSTAMP(t, e) \
-    ((blockIdx.x < 4 && (t) < 64) ? (void)(g_kvp_ttrace[blockIdx.x][(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
+    ((kvp_trace_slot() >= 0 && (t) < 64) ? (void)(g_kvp_ttrace[kvp_trace_slot()][(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
 #else
 #define KVP_STAMP(i) ((void)0)
 #define KVP_TSTAMP(t, e) ((void)0)
@@ -91,7 +94,7 @@ struct Params {
     int nk, nv;          // K and V ring depths
     float scale2;        // log2(e) / sqrt(d)
     uint32_t q_bytes, k_bytes, v_bytes;
-    uint32_t off_q, off_k, off_v, off_lse, off_cw, off_bar;
+    uint32_t off_q, off_k, off_v, off_lse, off_cw, off_wpos, off_bar;
     int cw_stride;       // floats per epilogue warp of phase 0 row offsets
     float* score;
     float* s1;
@@ -195,63 +198,105 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32]) {
     return v[0];
 }
 
-// Phase 0, one 32-column chunk for one key per thread: v[i] is the key's raw logit
-// against query row (chunk column) i, masked to -inf where not visible. cw[0..31] are the
-// warp's running offsets of those rows (log2 units, shared memory). Returns, in lane L,
-// the warp's sum over its 32 keys of 2^(t - cw) for column L; on overflow (a logit far
-// above its row's offset) the offsets of the chunk are raised first and *lsum (lane L's
-// running sum of column L) rescaled to match.
-__device__ __forceinline__ float lse_chunk_t(const float (&v)[32], float* cw, float scale2,
-                                             float& lsum) {
-    const int lane = threadIdx.x & 31;
-    float e[32];
+// Rare paths of the epilogue (the first tile of a head, tiles holding window keys, a
+// ragged last chunk, logits overflowing their row's offset) live in non-inlined
+// functions that load their chunk from TMEM themselves, so that the steady-state loop
+// carries none of their code or registers.
+
+// 32 TMEM columns of this warp's lanes at taddr: v[e] is the thread's key against local
+// column cbase + e, masked to -inf past the group's ncols columns and, inside the window
+// (key offset jw > 0), for query rows before the key.
+__device__ __forceinline__ void load_masked(uint32_t taddr, float (&v)[32], int cbase, int ncols,
+                                            int col0, int jw, const uint16_t* wpos) {
+    __syncwarp();
+    ptx::tmem_ld_32x32b_x32(taddr, v);
+    ptx::tmem_ld_wait(v);
 #pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-        const float4 c4 = *(const float4*)(cw + i);
-        e[i + 0] = ptx::ex2(fmaf(v[i + 0], scale2, -c4.x));
-        e[i + 1] = ptx::ex2(fmaf(v[i + 1], scale2, -c4.y));
-        e[i + 2] = ptx::ex2(fmaf(v[i + 2], scale2, -c4.z));
-        e[i + 3] = ptx::ex2(fmaf(v[i + 3], scale2, -c4.w));
+    for (int e = 0; e < 32; ++e) {
+        const int n = cbase + e;
+        if (n >= ncols || (jw > 0 && jw > (int)wpos[col0 + n])) v[e] = -INFINITY;
     }
-    float sum = warp_reduce_scatter32<false>(e);
-    if (__any_sync(0xffffffffu, !(sum < INFINITY))) {
-        // rare: raise each column's offset to the column's maximum where that is higher
+}
+
+// Phase 0, one chunk on the rare path. cw[0..31]: the warp's offsets (log2 units) of the
+// chunk's rows; `first` sets them to each row's maximum over the warp's keys. Returns
+// (lane L's sum of 2^(t - cw) over the warp's keys for row L of the chunk, lsum rescaled
+// if the offsets had to be raised to keep the exponentials finite).
+__device__ __forceinline__ float2 lse_chunk_slow(uint32_t taddr, int cbase, int ncols, int col0,
+                                              int jw, bool first, float* cw,
+                                              const uint16_t* wpos, float scale2, float lsum) {
+    const int lane = threadIdx.x & 31;
+    float v[32];
+    load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
+    if (first) {
+        const float cmax = warp_reduce_scatter32<true>(v);
+        __syncwarp();
+        cw[lane] = cmax == -INFINITY ? -1e30f : cmax * scale2;
+        __syncwarp();
+        load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
+    }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) e[i] = fmaf(v[i], scale2, -cw[i]);
-        float d = warp_reduce_scatter32<true>(e);
+    for (int i = 0; i < 32; ++i) v[i] = ptx::ex2(fmaf(v[i], scale2, -cw[i]));
+    float sum = warp_reduce_scatter32<false>(v);
+    if (__any_sync(0xffffffffu, !(sum < INFINITY))) {
+        load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = fmaf(v[i], scale2, -cw[i]);
+        float d = warp_reduce_scatter32<true>(v);
         d = d > 0.f ? d : 0.f;                    // also maps NaN (all masked) to 0
         lsum *= ptx::ex2(-d);
         __syncwarp();
         cw[lane] += d;
         __syncwarp();
+        load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) e[i] = ptx::ex2(fmaf(v[i], scale2, -cw[i]));
-        sum = warp_reduce_scatter32<false>(e);
+        for (int i = 0; i < 32; ++i) v[i] = ptx::ex2(fmaf(v[i], scale2, -cw[i]));
+        sum = warp_reduce_scatter32<false>(v);
     }
-    return sum;
+    return make_float2(sum, lsum);
 }
 
-// Phase 1, one 32-column chunk of one key: add 2^(t - lse2[n]) over the chunk's valid
-// query rows n = n0 + e (n < nend; inside the window, key offset jw <= n mod w).
-__device__ __forceinline__ void s1_chunk(const float (&v)[32], bool fast, int n0, int nend,
-                                         int jw, int w, const float* lse2, float scale2,
-                                         float& a0, float& a1, float& a2, float& a3) {
-    if (fast) {
+// Phase 0 hot path, one full chunk already in v (overwritten): lane L gets the warp's sum
+// of 2^(t - cw) for row L of the chunk; +inf or NaN tells the caller to take the rare path.
+__device__ __forceinline__ float lse_chunk_fast(float (&v)[32], const float* cw, float scale2) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-            const float4 l4 = *(const float4*)(lse2 + n0 + e);
-            a0 += ptx::ex2(fmaf(v[e + 0], scale2, -l4.x));
-            a1 += ptx::ex2(fmaf(v[e + 1], scale2, -l4.y));
-            a2 += ptx::ex2(fmaf(v[e + 2], scale2, -l4.z));
-            a3 += ptx::ex2(fmaf(v[e + 3], scale2, -l4.w));
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const int n = n0 + e;
-            if (n < nend && jw <= n % w) a0 += ptx::ex2(fmaf(v[e], scale2, -lse2[n]));
-        }
+    for (int i = 0; i < 32; i += 4) {
+        const float4 c4 = *(const float4*)(cw + i);
+        v[i + 0] = ptx::ex2(fmaf(v[i + 0], scale2, -c4.x));
+        v[i + 1] = ptx::ex2(fmaf(v[i + 1], scale2, -c4.y));
+        v[i + 2] = ptx::ex2(fmaf(v[i + 2], scale2, -c4.z));
+        v[i + 3] = ptx::ex2(fmaf(v[i + 3], scale2, -c4.w));
     }
+    return warp_reduce_scatter32<false>(v);
+}
+
+// Phase 1 hot path, one full chunk: add 2^(t - lse2[n0 + e]) over its 32 query rows.
+__device__ __forceinline__ void s1_chunk_fast(const float (&v)[32], const float* lse2, float scale2,
+                                              float& a0, float& a1, float& a2, float& a3) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+        const float4 l4 = *(const float4*)(lse2 + e);
+        a0 += ptx::ex2(fmaf(v[e + 0], scale2, -l4.x));
+        a1 += ptx::ex2(fmaf(v[e + 1], scale2, -l4.y));
+        a2 += ptx::ex2(fmaf(v[e + 2], scale2, -l4.z));
+        a3 += ptx::ex2(fmaf(v[e + 3], scale2, -l4.w));
+    }
+}
+
+// Phase 1 rare path, one chunk loaded and masked here: the chunk's part of the key's S1.
+__device__ __forceinline__ float s1_chunk_slow(uint32_t taddr, int cbase, int ncols, int col0, int jw,
+                                            const uint16_t* wpos, const float* lse2, float scale2) {
+    float v[32];
+    load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        // masked entries (past the group's columns, or not visible) contribute nothing
+        const int n = col0 + cbase + e;
+        if (v[e] != -INFINITY) a0 += ptx::ex2(fmaf(v[e], scale2, -lse2[n]));
+        if (v[e + 1] != -INFINITY) a1 += ptx::ex2(fmaf(v[e + 1], scale2, -lse2[n + 1]));
+    }
+    return a0 + a1;
 }
 
 }  // namespace
@@ -274,6 +319,8 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     // phase 0: [8 warps][cw_stride] row offsets; at the end of a head the same bytes stage
     // the warps' (offset, sum) pairs as float2 [8][cw_stride]
     float* cw_all = (float*)(smem + p.off_cw);
+    // window position i of query row n (row n = g * w + i), so no division in the loops
+    uint16_t* wpos = (uint16_t*)(smem + p.off_wpos);
     SmemBars* sb = (SmemBars*)(smem + p.off_bar);
 
     constexpr int kHalves = D / 64;                 // 128-byte swizzle rows per operand row
@@ -285,6 +332,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const long long T = p.total_tiles;
     const long long t0 = run_begin(blockIdx.x, T, p.grid), t1 = run_begin(blockIdx.x + 1, T, p.grid);
 
+    for (int n = threadIdx.x; n < p.rows; n += kThreads) wpos[n] = (uint16_t)(n % p.w);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxStages; ++s) {
             ptx::mbar_init(&sb->kfull[s], 1);
@@ -510,30 +558,47 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     const int j = key0 + lrow;                       // this thread's key
                     const bool full = key0 + kTile - 1 <= window0;
                     const int jw = j - window0;                      // > 0 only inside the window
-                    // one 32-column chunk: mask, (first tile) set offsets, fold into lw
+                    // masks, needed only by warps holding window keys and by a ragged last chunk
+                    auto mask_chunk = [&](float (&v)[32], int c) {
+                        if (jw > 0) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (jw > (int)wpos[col0 + c * 32 + e]) v[e] = -INFINITY;
+                        }
+                        if ((c + 1) * 32 > ncols) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (c * 32 + e >= ncols) v[e] = -INFINITY;
+                        }
+                    };
                     auto chunk0 = [&](float (&v)[32], int c) {
-                        if (!full || (c + 1) * 32 > ncols) {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const int n = c * 32 + e;
-                                if (n >= ncols || jw > (col0 + n) % p.w) v[e] = -INFINITY;
-                            }
-                        }
+                        mask_chunk(v, c);
                         if (first_tile) {
-                            // offsets from this (first) tile: each row's maximum over the warp's keys
-                            float m[32];
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) m[e] = v[e];
-                            const float cmax = warp_reduce_scatter32<true>(m);
+                            // offsets of the head's first tile: the logits of the warp's first
+                            // key (any offset within ~100 of a row's maximum keeps every
+                            // exponential finite; farther ones are caught below)
                             __syncwarp();
-                            cwp[c * 32 + lane] = cmax == -INFINITY ? -1e30f : cmax * p.scale2;
+                            if (lane == 0) {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e)
+                                    cwp[c * 32 + e] = v[e] == -INFINITY ? -1e30f : v[e] * p.scale2;
+                            }
                             __syncwarp();
                         }
+                        float sum = lse_chunk_fast(v, cwp + c * 32, p.scale2);
                         float lcur = 0.f;              // lane L: running sum of column c*32+L
 #pragma unroll
                         for (int cc = 0; cc < 8; ++cc)
                             if (cc == c) lcur = lw[cc];
-                        lcur += lse_chunk_t(v, cwp + c * 32, p.scale2, lcur);
+                        if (__any_sync(0xffffffffu, !(sum < INFINITY))) {
+                            // rare: a logit far above its row's offset; raise offsets, redo
+                            const float2 r = lse_chunk_slow(tstage + c * 32, c * 32, ncols, col0,
+                                                            jw, false, cwp + c * 32, wpos,
+                                                            p.scale2, lcur);
+                            sum = r.x;
+                            lcur = r.y;
+                        }
+                        lcur += sum;
 #pragma unroll
                         for (int cc = 0; cc < 8; ++cc)
                             if (cc == c) lw[cc] = lcur;
@@ -713,29 +778,34 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     const int jw = j - window0;                     // > 0 only inside the window
                     const int col0 = (p.split && wg == 1) ? p.n1 : 0;        // first query row
                     const int ncols = p.split ? (wg == 0 ? p.n1 : p.rows - p.n1) : p.rows;
-                    const int nch = (ncols + 31) >> 5;
                     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                    float x[32], y[32];
-                    __syncwarp();
-                    ptx::tmem_ld_32x32b_x32(tstage, x);
-                    ptx::tmem_ld_wait(x);
-                    for (int c = 0; c < nch; c += 2) {
-                        const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
-                        if (has1) {
-                            __syncwarp();
-                            ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
-                        }
-                        s1_chunk(x, full && (c + 1) * 32 <= ncols, col0 + c * 32, col0 + ncols, jw, p.w,
-                                 lse2, p.scale2, a0, a1, a2, a3);
-                        if (has1) {
-                            ptx::tmem_ld_wait(y);
-                            if (has2) {
+                    // the path is chosen per warp: TMEM loads are warp-collective
+                    if (__any_sync(0xffffffffu, jw > 0) || (ncols & 31)) {
+                        // window keys or a ragged last chunk: masked, chunk by chunk
+                        for (int c = 0; c < nch; ++c)
+                            a0 += s1_chunk_slow(tstage + c * 32, c * 32, ncols, col0, jw, wpos, lse2,
+                                                p.scale2);
+                    } else {
+                        float x[32], y[32];
+                        __syncwarp();
+                        ptx::tmem_ld_32x32b_x32(tstage, x);
+                        ptx::tmem_ld_wait(x);
+                        for (int c = 0; c < nch; c += 2) {
+                            const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
+                            if (has1) {
                                 __syncwarp();
-                                ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
+                                ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
                             }
-                            s1_chunk(y, full && (c + 2) * 32 <= ncols, col0 + (c + 1) * 32, col0 + ncols, jw,
-                                     p.w, lse2, p.scale2, a0, a1, a2, a3);
-                            if (has2) ptx::tmem_ld_wait(x);
+                            s1_chunk_fast(x, lse2 + col0 + c * 32, p.scale2, a0, a1, a2, a3);
+                            if (has1) {
+                                ptx::tmem_ld_wait(y);
+                                if (has2) {
+                                    __syncwarp();
+                                    ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
+                                }
+                                s1_chunk_fast(y, lse2 + col0 + (c + 1) * 32, p.scale2, a0, a1, a2, a3);
+                                if (has2) ptx::tmem_ld_wait(x);
+                            }
                         }
                     }
                     ptx::tc_fence_before();
@@ -882,7 +952,8 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     // lse2[rows] (16-byte padded), then the split-mode handoff comb[2][128]
     const size_t lse_floats = (size_t)((plan.rows + 3) / 4 * 4);
     const size_t lse_bytes = (lse_floats + (p.split ? 2 * kTile : 0)) * sizeof(float);
-    const size_t fixed = lse_bytes + cw_bytes + kBarBytes + 1024;
+    const size_t wpos_bytes = (size_t)((plan.rows + 7) / 8 * 8) * sizeof(uint16_t);
+    const size_t fixed = std::max(lse_bytes, cw_bytes) + wpos_bytes + kBarBytes + 1024;
     size_t total = 0;
     bool fit = false;
     for (auto& c : choices) {
@@ -899,9 +970,12 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.off_q = 0;
     p.off_k = qbytes;
     p.off_v = p.off_k + p.nk * tile_bytes;
-    p.off_lse = p.off_v + p.nv * tile_bytes;
-    p.off_cw = p.off_lse + (uint32_t)lse_bytes;
-    p.off_bar = p.off_cw + (uint32_t)cw_bytes;
+    // phase 0's row offsets / staging and phase 1's lse2 + handoff are never live at the
+    // same time (all epilogue threads pass a rendezvous between the phases): one region
+    p.off_cw = p.off_v + p.nv * tile_bytes;
+    p.off_lse = p.off_cw;
+    p.off_wpos = p.off_cw + (uint32_t)std::max(lse_bytes, cw_bytes);
+    p.off_bar = p.off_wpos + (uint32_t)wpos_bytes;
     static_assert(sizeof(SmemBars) <= kBarBytes, "barrier block");
     L->grid = p.grid;
     L->smem = std::max(total, (size_t)kMinSmem);
