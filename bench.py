@@ -221,6 +221,29 @@ def run_reference(a, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def rank_layer(rank):
+    """The layer (and so the seed) a rank evicts: every rank its own, independent unit
+    of work, so no data crosses between ranks."""
+    return rank
+
+
+def max_over_ranks(x, device, world):
+    """Max of a host float over all ranks (the slowest rank sets a multi-GPU time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_layer(elapsed_ms, steps, world):
+    """Whole-job time per layer: every rank evicts one layer per step, so the job
+    processes steps * world layers in the slowest rank's elapsed time."""
+    return elapsed_ms / (steps * world)
+
+
 def workload_config(wl, l2_note):
     return {"workload": wl.name, "batch": wl.batch, "hq": wl.hq, "hkv": wl.hkv,
             "head_dim": wl.head_dim, "seq_len": wl.seq_len, "window": wl.window,
@@ -247,7 +270,7 @@ def run_kvp(a, world, rank, local):
             dist.barrier()
 
     wl = synth.WORKLOADS[a.workload]
-    inp = synth.make_inputs(wl, layer=rank)        # every rank evicts its own layer
+    inp = synth.make_inputs(wl, layer=rank_layer(rank))   # every rank its own layer
     sh = kvp.make_shape(*wl.shape_tuple())
     to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
     q0, k0, v0 = to_dev(inp.q_win), to_dev(inp.k), to_dev(inp.v)
@@ -296,13 +319,8 @@ def run_kvp(a, world, rank, local):
         per_call["kvp_select"].append(e[1].elapsed_time(e[2]))
         per_call["kvp_compact"].append(e[2].elapsed_time(e[3]))
     mean_call = {k: float(np.mean(v)) for k, v in per_call.items()}
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-        ts = torch.tensor([mean_call["kvp_score"]], device=dev)
-        dist.all_reduce(ts, op=dist.ReduceOp.MAX)
-        mean_call["kvp_score"] = float(ts.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev, world)
+    mean_call["kvp_score"] = max_over_ranks(mean_call["kvp_score"], dev, world)
 
     # ---- end to end through the public API: host inputs in, host results out -------------
     hq = torch.from_numpy(inp.q_win.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -338,11 +356,7 @@ def run_kvp(a, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
 
     # result sanity on the last e2e step (cheap checks; parity lives in the tests)
     idx_np = h_idx.numpy()
@@ -351,8 +365,7 @@ def run_kvp(a, world, rank, local):
     line = None
     if rank == 0:
         peak, peak_kind = measured_peaks()
-        layers = a.steps * world
-        ms_per_layer = elapsed_ms / layers
+        ms_per_layer = job_ms_per_layer(elapsed_ms, a.steps, world)
         bytes_layer = wl.bytes_per_layer()
         score_bytes = bytes_layer["score"]
         achieved = score_bytes / (mean_call["kvp_score"] * 1e-3) / 1e9
@@ -373,7 +386,7 @@ def run_kvp(a, world, rank, local):
                          "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic_from_profile(srcs),
                          "algorithmic_bytes_per_launch": score_bytes},
-            "e2e": {"value": e2e_ms / e2e_steps / world * 1.0, "unit": "ms/layer",
+            "e2e": {"value": job_ms_per_layer(e2e_ms, e2e_steps, world), "unit": "ms/layer",
                     "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": a.steps * kvp.KERNELS_PER_LAYER,
             "clocks": clocks.summary(),
