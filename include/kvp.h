@@ -108,6 +108,31 @@ KVP_API kvp_status kvp_select(const kvp_shape* shape, const float* score, int32_
 KVP_API kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
                                const int32_t* idx, uint16_t* k_out, uint16_t* v_out, void* stream);
 
+/*
+ * kvp_score without a workspace, for callers that cannot allocate device memory at the
+ * time they evict: a serving engine that reserved the device for its own memory pool at
+ * start-up, code that may not allocate after initialisation, or a runtime that only
+ * passes in tensors it already owns. (The eviction method has no counterpart to this
+ * call; it is a deployment convenience.)
+ *
+ * Inputs, outputs and results are those of kvp_score. The scratch is a fixed array of
+ * KVP_STATIC_SCRATCH_BYTES bytes of device memory defined inside the library; every GPU
+ * that loads the library holds it until the process exits. A shape whose
+ * kvp_workspace_bytes() exceeds KVP_STATIC_SCRATCH_BYTES is rejected with
+ * KVP_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address (once per
+ *     device); make that first call before any stream capture on that device.
+ *   - All calls share the one array: calls that may overlap on the GPU (other streams,
+ *     other host threads, concurrent graphs) race and must be serialised by the caller.
+ *     Each call clears the parts of the array that must start at zero.
+ *   - The call allocates nothing (no cudaMalloc, no allocating library routine).
+ */
+#define KVP_STATIC_SCRATCH_BYTES ((size_t)2 << 20)
+
+KVP_API kvp_status kvp_score_static(const kvp_shape* shape, const uint16_t* q_win,
+                                    const uint16_t* k, const uint16_t* v, float* score,
+                                    float* s1, float* s2, void* stream);
+
 /* The name of the CUDA error behind the calling thread's most recent KVP_ERR_CUDA
  * ("cudaSuccess" if there was none). Host-only; never fails. */
 KVP_API const char* kvp_last_cuda_error(void);

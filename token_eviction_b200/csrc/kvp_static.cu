@@ -1,0 +1,74 @@
+// kvp_score_static: the scoring call with its scratch memory built into the library.
+//
+// Some callers cannot allocate device memory when they evict: a serving engine that
+// reserves the whole device for its own memory pool at start-up (a later cudaMalloc
+// fails or fragments the pool), code running where allocation is forbidden after
+// initialisation, or a host runtime that hands this library only the tensors it owns.
+// For them this entry point takes the same inputs and outputs as kvp_score but no
+// workspace: the scratch lives in a fixed-size array in device memory that the library
+// defines, which every GPU that loads the library keeps until the process exits.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "kvp.h"
+#include "kvp_internal.cuh"
+
+namespace kvp {
+namespace {
+
+// Largest scratch a shape may need here (its kvp_workspace_bytes); bigger shapes are
+// rejected with KVP_ERR_WORKSPACE. 2 MiB covers e.g. b1 x 32/8 heads at L = 128K and
+// b8 x 28/4 heads at L = 16K.
+constexpr size_t kStaticScratchBytes = KVP_STATIC_SCRATCH_BYTES;
+
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per device
+// (the array's name is only a host-side stand-in, not a device address).
+cudaError_t scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = ptr;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace kvp
+
+using namespace kvp;
+
+extern "C" kvp_status kvp_score_static(const kvp_shape* shape, const uint16_t* q_win,
+                                       const uint16_t* k, const uint16_t* v, float* score,
+                                       float* s1, float* s2, void* stream) {
+    if (!shape || !q_win || !k || !v || !score) return KVP_ERR_NULL;
+    Plan p;
+    if (!plan_of(*shape, &p)) return KVP_ERR_SHAPE;
+    auto a16 = [](const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; };
+    if (!a16(q_win) || !a16(k) || !a16(v) || !a16(score) || !a16(s1) || !a16(s2))
+        return KVP_ERR_ALIGN;
+    if (p.bytes > kStaticScratchBytes) return KVP_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    cudaError_t e = scratch_address(&scratch);
+    if (e == cudaSuccess)
+        e = launch_score(*shape, p, q_win, k, v, scratch, score, s1, s2, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return KVP_ERR_CUDA;
+    }
+    return KVP_OK;
+}
