@@ -42,12 +42,19 @@ bool plan_of(const kvp_shape& s, Plan* p) {
     const long long T = units * p->tiles_per_head;
     if (T > INT32_MAX) return false;
     p->total_tiles = (int)T;
-    p->grid = (int)std::min<long long>(kPlanGrid, T);
+    const long long tph = p->tiles_per_head;
+    const long long flat_grid = std::min<long long>(kPlanGrid, T);
+    const long long cph = units <= kPlanGrid ? std::min<long long>(kPlanGrid / units, tph) : 0;
+    // head-aligned runs unless their longest run exceeds the flat cut's by more than
+    // what a change of head costs a flat run
+    const bool aligned = cph > 0 && (tph + cph - 1) / cph <= (T + flat_grid - 1) / flat_grid + kHeadSwitchTiles;
+    p->cph = aligned ? (int)cph : 0;
+    p->grid = aligned ? (int)(cph * units) : (int)flat_grid;
     int slots = 0;
     for (long long h = 0; h < units; ++h) {
-        const long long f = h * p->tiles_per_head;
-        slots = std::max(slots, owner_of(f + p->tiles_per_head - 1, T, p->grid) -
-                                    owner_of(f, T, p->grid) + 1);
+        const long long f = h * tph;
+        slots = std::max(slots, owner_of(f + tph - 1, T, p->grid, tph, p->cph) -
+                                    owner_of(f, T, p->grid, tph, p->cph) + 1);
     }
     p->maxslots = slots * kSlotsPerCta;
     size_t off = 0;

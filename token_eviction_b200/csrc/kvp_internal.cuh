@@ -15,13 +15,16 @@ constexpr int kMaxGroupRows = 512;
 // How a shape is cut into work: 128-key tiles of the flattened (sequence, KV head, key)
 // space dealt out in contiguous runs to the scoring kernel's CTAs, and the workspace
 // layout. A pure function of the shape, so kvp_workspace_bytes, kvp_score and
-// kvp_select agree.
+// kvp_select agree. Runs are either aligned to the KV heads (every head cut into cph
+// runs of its own, so no CTA pays for a change of head) or, when that would leave too
+// many SMs idle, the flattened tiles cut evenly across all CTAs (cph = 0).
 struct Plan {
     int G;               // query heads per KV head
     int rows;            // G * w: window queries per KV head
     int tiles_per_head;  // 128-key tiles per (sequence, KV head)
     int total_tiles;     // over all (sequence, KV head)
     int grid;            // CTAs of the scoring kernel (one per SM, at most one per tile)
+    int cph;             // runs per KV head when runs are head-aligned; 0: flat runs
     int maxslots;        // partial-softmax slots per query row (CTAs touching one head)
     size_t off_done;     // uint32 per (sequence, KV head): CTAs done with phase 0
     size_t off_err;      // int: first device-side error code (0 = none)
@@ -39,14 +42,27 @@ constexpr int kSlotsPerCta = 1;
 
 bool plan_of(const kvp_shape& s, Plan* p);
 
-// The CTA whose run holds tile t when T tiles are cut into `grid` contiguous runs
-// [floor(c T / grid), floor((c + 1) T / grid)).
-__host__ __device__ __forceinline__ int owner_of(long long t, long long T, long long grid) {
-    return (int)(((t + 1) * grid + T - 1) / T - 1);
-}
-__host__ __device__ __forceinline__ long long run_begin(long long c, long long T, long long grid) {
+// Runs of the scoring kernel's CTAs over the T tiles (tph per KV head). Flat (cph = 0):
+// CTA c takes [floor(c T / grid), floor((c + 1) T / grid)). Head-aligned (cph > 0,
+// grid = cph * heads): CTA c takes part c % cph of head c / cph, the same cut within the
+// head's tph tiles.
+__host__ __device__ __forceinline__ long long run_begin(long long c, long long T, long long grid,
+                                                        long long tph, long long cph) {
+    if (cph > 0) return (c / cph) * tph + (c % cph) * tph / cph;
     return c * T / grid;
 }
+// The CTA whose run holds tile t.
+__host__ __device__ __forceinline__ int owner_of(long long t, long long T, long long grid,
+                                                 long long tph, long long cph) {
+    if (cph > 0) return (int)((t / tph) * cph + ((t % tph + 1) * cph + tph - 1) / tph - 1);
+    return (int)(((t + 1) * grid + T - 1) / T - 1);
+}
+
+// Tiles by which a head-aligned cut's longest run may exceed the flat cut's and still be
+// chosen. Measured on the 32K layer (8 heads, 148 SMs), 15-tile head-aligned runs were
+// slower than 14-tile flat runs with one change of head, so the aligned cut is taken only
+// where it is no longer (short contexts, where a flat run would span many heads).
+constexpr int kHeadSwitchTiles = 0;
 
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_score(const kvp_shape& s, const Plan& p, const uint16_t* q, const uint16_t* k,

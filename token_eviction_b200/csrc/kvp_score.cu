@@ -8,27 +8,29 @@
 // Window query i sits at position L - w + i and sees keys j <= L - w + i.
 //
 // The softmax denominators must be known before any key's S1 can be summed, so K is
-// swept twice; both sweeps run inside one kernel:
+// swept twice; both sweeps run inside one kernel. In both, tcgen05 computes the tile's
+// logits transposed, D[key, row] = K_tile[key] . Q_group[row] (M = 128 keys, N = G w
+// query rows), so every epilogue thread owns one key and each TMEM column is a query row.
 //   phase 0 (log-sum-exp): each CTA owns a contiguous run of 128-key tiles of the
-//     flattened (sequence, KV head, tile) space. Per tile, tcgen05 computes the logits
-//     D[row, key] = Q_group[row] . K_tile[key] (M = query rows, N = 128 keys) into TMEM;
-//     the epilogue keeps, per query row, a running max m and sum l of 2^(t - m),
-//     t = logit * log2(e) / sqrt(d). At the end of each KV head in its run, a CTA
-//     publishes (m, l) per row into its slots and bumps the head's completion counter.
+//     flattened (sequence, KV head, tile) space. Per query row, each warp keeps a running
+//     offset and sum of 2^(t - offset) over its 32 keys, t = logit * log2(e) / sqrt(d);
+//     a butterfly reduce-scatter turns a 32 x 32 chunk of exponentials into per-row sums.
+//     At the end of each KV head in its run, a CTA combines its warps' (offset, sum)
+//     pairs, publishes one slot per row and bumps the head's completion counter.
 //   phase 1 (scores): the same CTA sweeps the same tiles again (K now mostly from L2).
 //     Before its first tile of a head it waits (bounded) until every CTA touching that
 //     head has published, then merges the slots into lse2 = M + log2(sum_s l_s 2^(m_s - M))
-//     per row. Per tile, tcgen05 computes the transposed logits D[key, row] (M = 128
-//     keys, N = G w rows), so each epilogue thread owns one key and sums 2^(t - lse2)
-//     over the row's TMEM columns with no cross-thread reduction; the key's V row is
-//     read once from shared memory for S2, and S (and S1, S2 if asked) is written.
-// Warp roles: warp 0 issues TMA loads (K ring, V ring, the group's query rows), warp 1
+//     per row. Per tile each thread sums 2^(t - lse2) over its key's row columns, reads
+//     the key's V row once from shared memory for S2, and writes S (and S1, S2 if asked).
+// Loads go through a ring of tile slots in shared memory: phase 0 streams K through all
+// of them; phase 1 gives V (from HBM) the larger share and K (mostly L2) the rest.
+// Warp roles: warp 0 issues TMA loads (the ring and the group's query rows), warp 1
 // allocates TMEM and issues the MMAs from one thread, and two epilogue warpgroups
-// (warps 2-5 and 6-9, one TMEM lane quarter per warp) each own one of two TMEM
-// accumulator stages. When a tile's accumulator fits one stage (G w <= 256) the groups
-// take alternate tiles; otherwise every tile is split across both stages (query-row
-// halves in phase 0, column halves in phase 1) and the second group hands its partial
-// S1 to the first through shared memory.
+// (warps 2-5 and 6-9, one TMEM lane quarter per warp) each own TMEM accumulator
+// stages. When a tile's accumulator fits one stage (G w <= 256) the groups take
+// alternate tiles; otherwise every tile is split across both stages (query-row halves in
+// phase 0, column halves in phase 1) and the second group hands its partial S1 to the
+// first through shared memory.
 // Every wait is bounded by a timer; a wait that gives up records an error code in the
 // workspace and the CTA unwinds without touching TMEM or shared memory still in use.
 #include <cuda.h>
@@ -51,7 +53,7 @@ constexpr int kTile = 128;                        // keys per tile
 constexpr int kEpiGroups = 2;                     // epilogue warpgroups
 constexpr int kEpiThreads = 128 * kEpiGroups;
 constexpr int kThreads = 64 + kEpiThreads;        // + TMA warp + MMA warp
-constexpr int kMaxStages = 4;
+constexpr int kMaxSlots = 8;                     // tile slots of the load ring
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kMaxStageCols = 256;           // widest accumulator stage
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s on any single wait
@@ -90,11 +92,11 @@ struct Params {
     int split;           // 0: groups alternate tiles; 1: every tile split over both stages
     int stage_cols;      // TMEM columns per accumulator stage (128 or 256)
     int spg;             // accumulator stages per epilogue group (2 when a stage is 128 wide)
-    int tiles_per_head, total_tiles, grid, maxslots;
-    int nk, nv;          // K and V ring depths
+    int tiles_per_head, total_tiles, grid, cph, maxslots;
+    int ns, nk1, nv1;    // ring slots; phase 1 gives K slots [0, nk1), V slots [nk1, ns)
     float scale2;        // log2(e) / sqrt(d)
     uint32_t q_bytes, k_bytes, v_bytes;
-    uint32_t off_q, off_k, off_v, off_lse, off_cw, off_wpos, off_bar;
+    uint32_t off_q, off_slots, off_lse, off_cw, off_wpos, off_bar;
     int cw_stride;       // floats per epilogue warp of phase 0 row offsets
     float* score;
     float* s1;
@@ -105,8 +107,8 @@ struct Params {
 };
 
 struct SmemBars {
-    uint64_t kfull[kMaxStages], kempty[kMaxStages];
-    uint64_t vfull[kMaxStages], vempty[kMaxStages];
+    uint64_t kfull[kMaxSlots], kempty[kMaxSlots];   // per slot, for its K loads
+    uint64_t vfull[kMaxSlots], vempty[kMaxSlots];   // per phase 1 V slot (index s - nk1)
     uint64_t accfull[4], accempty[4];
     uint64_t combfull[2], combempty[2];
     uint64_t qfull, qempty, fin;
@@ -132,6 +134,14 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemB
             return false;
         }
     }
+}
+
+// Wait for phase `parity` of `bar` for at most the wait limit, whatever the CTA's state:
+// used before exit, so that no copy is still writing this CTA's shared memory.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait(bar, parity))
+        if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) return;
 }
 
 // Rendezvous of all epilogue threads on an mbarrier, so that a thread that gives up a
@@ -161,6 +171,23 @@ __device__ __forceinline__ int acc_stage(int split, int spg, int i, int g, uint3
     const int u = i >> 1;
     parity = (uint32_t)(u / spg) & 1u;
     return g + 2 * (u % spg);
+}
+
+// The load ring. Phase 0 streams only K, through all ns slots in turn; phase 1 streams K
+// through slots [0, nk1) and V through slots [nk1, ns). Each slot's K loads are counted
+// across both phases, so the parity of a slot's barriers follows from the tile number.
+__device__ __forceinline__ int ring_uses(int s, int period, int n) {   // uses of slot s
+    return n > s ? (n - s + period - 1) / period : 0;                   // among n tiles
+}
+// K slot of the run's tile i in `phase`, and the number of that slot's earlier K loads.
+__device__ __forceinline__ int k_slot(int phase, int i, int n, const Params& p, int& use) {
+    if (phase == 0) {
+        use = i / p.ns;
+        return i % p.ns;
+    }
+    const int s = i % p.nk1;
+    use = ring_uses(s, p.ns, n) + i / p.nk1;
+    return s;
 }
 
 // Segments of a CTA's run: maximal stretches of tiles within one KV head.
@@ -198,10 +225,10 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32]) {
     return v[0];
 }
 
-// Rare paths of the epilogue (the first tile of a head, tiles holding window keys, a
-// ragged last chunk, logits overflowing their row's offset) live in non-inlined
-// functions that load their chunk from TMEM themselves, so that the steady-state loop
-// carries none of their code or registers.
+// Rare paths of the epilogue (tiles holding window keys, a ragged last chunk, logits
+// overflowing their row's offset) live in non-inlined functions that take only scalars
+// and load their chunk from TMEM themselves, so that the steady-state loops stay small
+// (the instruction cache holds them) and carry none of the rare paths' registers.
 
 // 32 TMEM columns of this warp's lanes at taddr: v[e] is the thread's key against local
 // column cbase + e, masked to -inf past the group's ncols columns and, inside the window
@@ -222,7 +249,7 @@ __device__ __forceinline__ void load_masked(uint32_t taddr, float (&v)[32], int 
 // chunk's rows; `first` sets them to each row's maximum over the warp's keys. Returns
 // (lane L's sum of 2^(t - cw) over the warp's keys for row L of the chunk, lsum rescaled
 // if the offsets had to be raised to keep the exponentials finite).
-__device__ __forceinline__ float2 lse_chunk_slow(uint32_t taddr, int cbase, int ncols, int col0,
+__device__ __noinline__ float2 lse_chunk_slow(uint32_t taddr, int cbase, int ncols, int col0,
                                               int jw, bool first, float* cw,
                                               const uint16_t* wpos, float scale2, float lsum) {
     const int lane = threadIdx.x & 31;
@@ -270,6 +297,25 @@ __device__ __forceinline__ float lse_chunk_fast(float (&v)[32], const float* cw,
     return warp_reduce_scatter32<false>(v);
 }
 
+// Phase 0 hot path, two full chunks at once (offsets cw[0..63]): each element becomes
+// 2^(t - cw) in place, the two chunks interleaved for independent work in flight.
+__device__ __forceinline__ void lse_pair_fast(float (&x)[32], float (&y)[32], const float* cw,
+                                              float scale2) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+        const float4 c4 = *(const float4*)(cw + i);
+        const float4 d4 = *(const float4*)(cw + 32 + i);
+        x[i + 0] = ptx::ex2(fmaf(x[i + 0], scale2, -c4.x));
+        x[i + 1] = ptx::ex2(fmaf(x[i + 1], scale2, -c4.y));
+        x[i + 2] = ptx::ex2(fmaf(x[i + 2], scale2, -c4.z));
+        x[i + 3] = ptx::ex2(fmaf(x[i + 3], scale2, -c4.w));
+        y[i + 0] = ptx::ex2(fmaf(y[i + 0], scale2, -d4.x));
+        y[i + 1] = ptx::ex2(fmaf(y[i + 1], scale2, -d4.y));
+        y[i + 2] = ptx::ex2(fmaf(y[i + 2], scale2, -d4.z));
+        y[i + 3] = ptx::ex2(fmaf(y[i + 3], scale2, -d4.w));
+    }
+}
+
 // Phase 1 hot path, one full chunk: add 2^(t - lse2[n0 + e]) over its 32 query rows.
 __device__ __forceinline__ void s1_chunk_fast(const float (&v)[32], const float* lse2, float scale2,
                                               float& a0, float& a1, float& a2, float& a3) {
@@ -284,7 +330,7 @@ __device__ __forceinline__ void s1_chunk_fast(const float (&v)[32], const float*
 }
 
 // Phase 1 rare path, one chunk loaded and masked here: the chunk's part of the key's S1.
-__device__ __forceinline__ float s1_chunk_slow(uint32_t taddr, int cbase, int ncols, int col0, int jw,
+__device__ __noinline__ float s1_chunk_slow(uint32_t taddr, int cbase, int ncols, int col0, int jw,
                                             const uint16_t* wpos, const float* lse2, float scale2) {
     float v[32];
     load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
@@ -312,8 +358,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* Qs = smem + p.off_q;
-    uint8_t* Ks = smem + p.off_k;
-    uint8_t* Vs = smem + p.off_v;
+    uint8_t* Slots = smem + p.off_slots;               // ring slots of tile_bytes each
     float* lse2 = (float*)(smem + p.off_lse);          // [rows, padded to 4]
     float* comb = lse2 + ((p.rows + 3) & ~3);           // [2][128] partial S1 handoff (split mode)
     // phase 0: [8 warps][cw_stride] row offsets; at the end of a head the same bytes stage
@@ -325,16 +370,17 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
     constexpr int kHalves = D / 64;                 // 128-byte swizzle rows per operand row
     constexpr uint32_t kHalfTile = kTile * 128;     // bytes of one 64-column half of a tile
-    const uint32_t kstage = kTile * D * 2, vstage = kTile * D * 2;
+    constexpr uint32_t kSlotBytes = kTile * D * 2;
     const uint32_t qhalf = (uint32_t)p.qrows * 128;  // bytes of one 64-column half of Q
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long T = p.total_tiles;
-    const long long t0 = run_begin(blockIdx.x, T, p.grid), t1 = run_begin(blockIdx.x + 1, T, p.grid);
+    const long long t0 = run_begin(blockIdx.x, T, p.grid, p.tiles_per_head, p.cph);
+    const long long t1 = run_begin(blockIdx.x + 1, T, p.grid, p.tiles_per_head, p.cph);
 
     for (int n = threadIdx.x; n < p.rows; n += kThreads) wpos[n] = (uint16_t)(n % p.w);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kMaxStages; ++s) {
+        for (int s = 0; s < kMaxSlots; ++s) {
             ptx::mbar_init(&sb->kfull[s], 1);
             ptx::mbar_init(&sb->kempty[s], 1);
             ptx::mbar_init(&sb->vfull[s], 1);
@@ -386,12 +432,15 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         if (lane == 0) {
             const uint64_t pol_keep = ptx::policy_evict_last();
             const uint64_t pol_stream = ptx::policy_evict_first();
-            int kit = 0, vit = 0, qgen = 0, cur = -1;
+            const int n = (int)(t1 - t0);
+            int qgen = 0, cur = -1;
+            int kiss[kMaxSlots] = {}, viss[kMaxSlots] = {};   // loads issued per slot
             bool ok = true;
             for (int phase = 0; phase < 2 && ok; ++phase) {
                 RunIter it(t0, t1, p.tiles_per_head);
                 int head;
                 long long a, b;
+                int i = 0;                                  // tile number within the run
                 while (ok && it.next(head, a, b)) {
                     if (head != cur) {
                         if (qgen > 0 && !(ok = wait_phase(&sb->qempty, (qgen - 1) & 1, sb, p.err, kErrWaitTma))) break;
@@ -404,48 +453,55 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         ++qgen;
                         cur = head;
                     }
-                    for (long long t = a; t < b; ++t) {
+                    for (long long t = a; t < b; ++t, ++i) {
                         const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
-                        const int s = kit % p.nk;
-                        if (!(ok = wait_phase(&sb->kempty[s], ((kit / p.nk) & 1) ^ 1, sb, p.err, kErrWaitTma))) break;
-                        KVP_TSTAMP(kit, 0);
+                        int use;
+                        const int s = k_slot(phase, i, n, p, use);
+                        if (!(ok = wait_phase(&sb->kempty[s], (use & 1) ^ 1, sb, p.err, kErrWaitTma))) break;
+                        KVP_TSTAMP(phase * n + i, 0);
                         ptx::mbar_arrive_expect_tx(&sb->kfull[s], p.k_bytes);
                         for (int c = 0; c < kHalves; ++c)
-                            ptx::tma_load_3d(Ks + s * kstage + c * kHalfTile, &kmap, &sb->kfull[s],
+                            ptx::tma_load_3d(Slots + s * kSlotBytes + c * kHalfTile, &kmap, &sb->kfull[s],
                                              c * 64, key0, head, phase == 0 ? pol_keep : pol_stream);
-                        ++kit;
+                        ++kiss[s];
                         if (phase == 1) {
-                            const int sv = vit % p.nv;
-                            if (!(ok = wait_phase(&sb->vempty[sv], ((vit / p.nv) & 1) ^ 1, sb, p.err, kErrWaitTma))) break;
-                            KVP_TSTAMP(kit - 1, 6);
-                            ptx::mbar_arrive_expect_tx(&sb->vfull[sv], p.v_bytes);
-                            ptx::tma_load_3d(Vs + sv * vstage, &vmap, &sb->vfull[sv], 0, key0, head,
+                            const int jv = i % p.nv1, sv = p.nk1 + jv, vuse = i / p.nv1;
+                            // a V slot's first load waits for its last K load of phase 0 to be consumed
+                            const int u0 = vuse == 0 ? ring_uses(sv, p.ns, n) : 0;
+                            if (u0 > 0 && !(ok = wait_phase(&sb->kempty[sv], (u0 - 1) & 1, sb, p.err, kErrWaitTma))) break;
+                            if (!(ok = wait_phase(&sb->vempty[jv], (vuse & 1) ^ 1, sb, p.err, kErrWaitTma))) break;
+                            KVP_TSTAMP(phase * n + i, 6);
+                            ptx::mbar_arrive_expect_tx(&sb->vfull[jv], p.v_bytes);
+                            ptx::tma_load_3d(Slots + sv * kSlotBytes, &vmap, &sb->vfull[jv], 0, key0, head,
                                              pol_stream);
-                            ++vit;
+                            ++viss[jv];
                         }
                     }
                 }
                 KVP_STAMP(1 + phase);
             }
-            // Never leave with copies in flight: wait for the last load of every stage.
-            for (int i = max(0, kit - p.nk); i < kit; ++i)
-                wait_phase(&sb->kfull[i % p.nk], (i / p.nk) & 1, sb, p.err, kErrWaitTma);
-            for (int i = max(0, vit - p.nv); i < vit; ++i)
-                wait_phase(&sb->vfull[i % p.nv], (i / p.nv) & 1, sb, p.err, kErrWaitTma);
-            if (qgen > 0) wait_phase(&sb->qfull, (qgen - 1) & 1, sb, p.err, kErrWaitTma);
+            // Never leave with copies in flight: wait for the last load issued to every slot
+            // (these waits do not stop early when the CTA unwinds).
+            for (int s2 = 0; s2 < p.ns; ++s2)
+                if (kiss[s2] > 0) drain_wait(&sb->kfull[s2], (kiss[s2] - 1) & 1);
+            for (int jv = 0; jv < p.nv1; ++jv)
+                if (viss[jv] > 0) drain_wait(&sb->vfull[jv], (viss[jv] - 1) & 1);
+            if (qgen > 0) drain_wait(&sb->qfull, (qgen - 1) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc1a = ptx::idesc_bf16_f32(128, p.n1);
             const uint32_t idesc1b = ptx::idesc_bf16_f32(128, p.n2 > 0 ? p.n2 : 16);
-            const uint32_t q_addr = ptx::smem_u32(Qs), k_addr = ptx::smem_u32(Ks);
-            int kit = 0, ait = 0, qgen = 0, cur = -1;
+            const uint32_t q_addr = ptx::smem_u32(Qs), k_addr = ptx::smem_u32(Slots);
+            const int n = (int)(t1 - t0);
+            int ait = 0, qgen = 0, cur = -1;
             bool ok = true;
             for (int phase = 0; phase < 2 && ok; ++phase) {
                 RunIter it(t0, t1, p.tiles_per_head);
                 int head;
                 long long a, b;
+                int i = 0;                                  // tile number within the run
                 while (ok && it.next(head, a, b)) {
                     if (head != cur) {
                         if (!(ok = wait_phase(&sb->qfull, qgen & 1, sb, p.err, kErrWaitMma))) break;
@@ -453,12 +509,15 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         cur = head;
                         ptx::tc_fence_after();
                     }
-                    for (long long t = a; t < b; ++t) {
-                        const int s = kit % p.nk;
-                        if (!(ok = wait_phase(&sb->kfull[s], (kit / p.nk) & 1, sb, p.err, kErrWaitMma))) break;
+                    for (long long t = a; t < b; ++t, ++i) {
+                        const int kit = phase * n + i;              // trace index
+                        (void)kit;
+                        int use;
+                        const int s = k_slot(phase, i, n, p, use);
+                        if (!(ok = wait_phase(&sb->kfull[s], use & 1, sb, p.err, kErrWaitMma))) break;
                         KVP_TSTAMP(kit, 1);
                         KVP_MSTAMP(kit, 0);
-                        const uint32_t kbase = k_addr + s * kstage;
+                        const uint32_t kbase = k_addr + s * kSlotBytes;
                         // stages written for this tile: one (alternating) or both (split)
                         const int g_lo = p.split ? 0 : (ait & 1);
                         const int g_hi = p.split ? 1 : (ait & 1);
@@ -496,7 +555,6 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         ptx::mma_commit(&sb->kempty[s]);
                         KVP_TSTAMP(kit, 3);
                         KVP_MSTAMP(kit, 11);
-                        ++kit;
                         ++ait;
                     }
                     if (!ok) break;
@@ -556,7 +614,6 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     ptx::tc_fence_after();
                     const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
                     const int j = key0 + lrow;                       // this thread's key
-                    const bool full = key0 + kTile - 1 <= window0;
                     const int jw = j - window0;                      // > 0 only inside the window
                     // masks, needed only by warps holding window keys and by a ragged last chunk
                     auto mask_chunk = [&](float (&v)[32], int c) {
@@ -604,24 +661,89 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                             if (cc == c) lw[cc] = lcur;
                     };
                     float x[32], y[32];
-                    __syncwarp();
-                    ptx::tmem_ld_32x32b_x32(tstage, x);
-                    ptx::tmem_ld_wait(x);
-                    for (int c = 0; c < nch; c += 2) {
-                        const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
-                        if (has1) {
+                    // the path is chosen per warp: TMEM loads are warp-collective
+                    if (__any_sync(0xffffffffu, jw > 0) || (ncols & 31) || (nch & 1)) {
+                        // window keys, a ragged last chunk or an odd chunk count: masked,
+                        // chunk by chunk
+                        __syncwarp();
+                        ptx::tmem_ld_32x32b_x32(tstage, x);
+                        ptx::tmem_ld_wait(x);
+                        for (int c = 0; c < nch; c += 2) {
+                            const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
+                            if (has1) {
+                                __syncwarp();
+                                ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
+                            }
+                            chunk0(x, c);
+                            if (has1) {
+                                ptx::tmem_ld_wait(y);
+                                if (has2) {
+                                    __syncwarp();
+                                    ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
+                                }
+                                chunk0(y, c + 1);
+                                if (has2) ptx::tmem_ld_wait(x);
+                            }
+                        }
+                    } else {
+                        // steady state: whole chunks, no masks; two chunks at a time so that
+                        // their exponentials and shuffles interleave. A head's first tile
+                        // takes its row offsets from the warp's first key on the way.
+                        __syncwarp();
+                        ptx::tmem_ld_32x32b_x32(tstage, x);
+                        ptx::tmem_ld_wait(x);
+#pragma unroll 1
+                        for (int c = 0; c < nch; c += 2) {
                             __syncwarp();
                             ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
-                        }
-                        chunk0(x, c);
-                        if (has1) {
                             ptx::tmem_ld_wait(y);
-                            if (has2) {
+                            if (first_tile) {
+                                __syncwarp();
+                                if (lane == 0) {
+#pragma unroll
+                                    for (int e = 0; e < 32; e += 4) {
+                                        *(float4*)(cwp + c * 32 + e) =
+                                            make_float4(x[e] * p.scale2, x[e + 1] * p.scale2,
+                                                        x[e + 2] * p.scale2, x[e + 3] * p.scale2);
+                                        *(float4*)(cwp + c * 32 + 32 + e) =
+                                            make_float4(y[e] * p.scale2, y[e + 1] * p.scale2,
+                                                        y[e + 2] * p.scale2, y[e + 3] * p.scale2);
+                                    }
+                                }
+                                __syncwarp();
+                            }
+                            lse_pair_fast(x, y, cwp + c * 32, p.scale2);
+                            float s0 = warp_reduce_scatter32<false>(x);
+                            float s1 = warp_reduce_scatter32<false>(y);
+                            float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+                            for (int cc = 0; cc < 8; cc += 2)
+                                if (cc == c) {
+                                    l0 = lw[cc];
+                                    l1 = lw[cc + 1];
+                                }
+                            if (__any_sync(0xffffffffu, !(s0 < INFINITY) || !(s1 < INFINITY))) {
+                                // rare: a logit far above its row's offset; raise, redo
+                                float2 r = lse_chunk_slow(tstage + c * 32, c * 32, ncols, col0, jw, false,
+                                                          cwp + c * 32, wpos, p.scale2, l0);
+                                s0 = r.x;
+                                l0 = r.y;
+                                r = lse_chunk_slow(tstage + (c + 1) * 32, (c + 1) * 32, ncols, col0, jw, false,
+                                                   cwp + (c + 1) * 32, wpos, p.scale2, l1);
+                                s1 = r.x;
+                                l1 = r.y;
+                            }
+#pragma unroll
+                            for (int cc = 0; cc < 8; cc += 2)
+                                if (cc == c) {
+                                    lw[cc] = l0 + s0;
+                                    lw[cc + 1] = l1 + s1;
+                                }
+                            if (c + 2 < nch) {
                                 __syncwarp();
                                 ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
+                                ptx::tmem_ld_wait(x);
                             }
-                            chunk0(y, c + 1);
-                            if (has2) ptx::tmem_ld_wait(x);
                         }
                     }
                     first_tile = false;
@@ -650,7 +772,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 }
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
                 const long long first = (long long)head * p.tiles_per_head;
-                const int slot = (int)blockIdx.x - owner_of(first, T, p.grid);
+                const int slot = (int)blockIdx.x - owner_of(first, T, p.grid, p.tiles_per_head, p.cph);
                 const int r0 = group_row0(head);
                 for (int r = et; r < p.rows; r += kEpiThreads) {
                     // warps holding row r: all eight, or the four of the group owning it
@@ -688,7 +810,8 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             int pt = 0;                                   // phase 1 tile counter (V ring, handoff)
             while (ok && it.next(head, a, b)) {
                 const long long first = (long long)head * p.tiles_per_head;
-                const int touch = owner_of(first + p.tiles_per_head - 1, T, p.grid) - owner_of(first, T, p.grid) + 1;
+                const int touch = owner_of(first + p.tiles_per_head - 1, T, p.grid, p.tiles_per_head, p.cph) -
+                                  owner_of(first, T, p.grid, p.tiles_per_head, p.cph) + 1;
                 // the previous head's lse2 is no longer in use
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
                 if (et == 0) {
@@ -749,10 +872,10 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     if (reads_v) {
                         // S2: max |V[j, :]| from the staged tile, 16-byte pieces in a
                         // rotated order per lane (conflict-free shared-memory reads)
-                        const int sv = pt % p.nv;
-                        if (!(ok = wait_phase(&sb->vfull[sv], (pt / p.nv) & 1, sb, p.err, kErrWaitEpi))) break;
+                        const int jv = pt % p.nv1;
+                        if (!(ok = wait_phase(&sb->vfull[jv], (pt / p.nv1) & 1, sb, p.err, kErrWaitEpi))) break;
                         if (lrow == 0) KVP_TSTAMP(ait, 7);
-                        const uint4* vrow = (const uint4*)(Vs + sv * vstage + lrow * (D * 2));
+                        const uint4* vrow = (const uint4*)(Slots + (p.nk1 + jv) * kSlotBytes + lrow * (D * 2));
                         constexpr int kPieces = D * 2 / 16;
                         uint32_t mx = 0;
 #pragma unroll
@@ -765,7 +888,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         }
                         s2v = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
                         __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&sb->vempty[sv]);
+                        if (lane == 0) ptx::mbar_arrive(&sb->vempty[jv]);
                     }
                     // S1 over this group's columns
                     uint32_t parity;
@@ -774,7 +897,6 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     if (!(ok = wait_phase(&sb->accfull[st], parity, sb, p.err, kErrWaitEpi))) break;
                     if (lrow == 0) KVP_TSTAMP(ait, 4);
                     ptx::tc_fence_after();
-                    const bool full = key0 + kTile - 1 <= window0;
                     const int jw = j - window0;                     // > 0 only inside the window
                     const int col0 = (p.split && wg == 1) ? p.n1 : 0;        // first query row
                     const int ncols = p.split ? (wg == 0 ? p.n1 : p.rows - p.n1) : p.rows;
@@ -919,14 +1041,17 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.spg = p.stage_cols == 128 ? 2 : 1;
     p.tiles_per_head = plan.tiles_per_head;
     p.total_tiles = plan.total_tiles;
-    p.grid = std::min(plan.grid, sms);
+    // the planned cut, or a flat cut over the SMs of a smaller device
+    p.cph = plan.grid <= sms ? plan.cph : 0;
+    p.grid = plan.grid <= sms ? plan.grid : sms;
     // slots each head needs with this grid must fit the workspace's
     {
         const long long T = p.total_tiles;
         int need = 0;
         for (int h = 0; h < s.batch * s.hkv; ++h) {
             const long long f = (long long)h * p.tiles_per_head;
-            need = std::max(need, owner_of(f + p.tiles_per_head - 1, T, p.grid) - owner_of(f, T, p.grid) + 1);
+            need = std::max(need, owner_of(f + p.tiles_per_head - 1, T, p.grid, p.tiles_per_head, p.cph) -
+                                      owner_of(f, T, p.grid, p.tiles_per_head, p.cph) + 1);
         }
         if (need * kSlotsPerCta > plan.maxslots) return false;
     }
@@ -944,35 +1069,33 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     const int group_cols = p.split ? std::max(p.n1, plan.rows - p.n1) : plan.rows;
     p.cw_stride = (group_cols + 31) / 32 * 32;
     const size_t cw_bytes = (size_t)(kEpiThreads / 32) * p.cw_stride * sizeof(float2);
-    // Alternate-tile mode: both epilogue groups read V stages, each its own tiles; with an
-    // even V ring a group only ever waits on its own stages, one phase ahead at most (an
-    // odd ring would make a group wait two phases ahead on a shared stage, where the
-    // parity test cannot tell the phases apart). Split mode: group 0 alone reads V.
-    const int choices[5][2] = {{4, 2}, {3, 2}, {2, 2}, {3, 1}, {2, 1}};
     // lse2[rows] (16-byte padded), then the split-mode handoff comb[2][128]
     const size_t lse_floats = (size_t)((plan.rows + 3) / 4 * 4);
     const size_t lse_bytes = (lse_floats + (p.split ? 2 * kTile : 0)) * sizeof(float);
     const size_t wpos_bytes = (size_t)((plan.rows + 7) / 8 * 8) * sizeof(uint16_t);
     const size_t fixed = std::max(lse_bytes, cw_bytes) + wpos_bytes + kBarBytes + 1024;
-    size_t total = 0;
-    bool fit = false;
-    for (auto& c : choices) {
-        total = qbytes + (size_t)(c[0] + c[1]) * tile_bytes + fixed;
-        if (!p.split && c[1] % 2 != 0) continue;
-        if (total <= (size_t)kSmemLimit) {
-            p.nk = c[0];
-            p.nv = c[1];
-            fit = true;
-            break;
-        }
+    // As many ring slots as fit. Phase 1 splits them between K (read again, mostly from
+    // L2) and V (from HBM, so it gets the deeper share). Alternate-tile mode: both epilogue
+    // groups read V slots, each its own tiles; with an even number of V slots a group only
+    // ever waits on its own slots, one phase ahead at most (an odd count would make a group
+    // wait two phases ahead on a shared slot, where the parity test cannot tell the phases
+    // apart). Split mode: group 0 alone reads V.
+    if (qbytes + fixed > (size_t)kSmemLimit) return false;
+    p.ns = (int)std::min<size_t>(kMaxSlots, ((size_t)kSmemLimit - qbytes - fixed) / tile_bytes);
+    if (p.split) {
+        if (p.ns < 2) return false;
+        p.nv1 = p.ns / 2;
+    } else {
+        if (p.ns < 3) return false;
+        p.nv1 = p.ns >= 6 ? 4 : 2;
     }
-    if (!fit) return false;
+    p.nk1 = p.ns - p.nv1;
+    const size_t total = qbytes + (size_t)p.ns * tile_bytes + fixed;
     p.off_q = 0;
-    p.off_k = qbytes;
-    p.off_v = p.off_k + p.nk * tile_bytes;
+    p.off_slots = qbytes;
     // phase 0's row offsets / staging and phase 1's lse2 + handoff are never live at the
     // same time (all epilogue threads pass a rendezvous between the phases): one region
-    p.off_cw = p.off_v + p.nv * tile_bytes;
+    p.off_cw = p.off_slots + p.ns * tile_bytes;
     p.off_lse = p.off_cw;
     p.off_wpos = p.off_cw + (uint32_t)std::max(lse_bytes, cw_bytes);
     p.off_bar = p.off_wpos + (uint32_t)wpos_bytes;
