@@ -2,6 +2,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <mutex>
+#include <vector>
 #include <cstdint>
 
 #include "kvp.h"
@@ -15,6 +17,34 @@ int num_sms() {
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
         return n;
     return 148;
+}
+
+cudaError_t allow_dynamic_smem(const void* func, size_t bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    struct Entry {
+        int dev;
+        const void* func;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> raised;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& r : raised)
+        if (r.dev == dev && r.func == func) return cudaSuccess;
+    int optin = 0;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return e;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, func)) != cudaSuccess) return e;
+    // the opt-in maximum covers static and dynamic shared memory together
+    const size_t max_dynamic = (size_t)optin > fa.sharedSizeBytes ? (size_t)optin - fa.sharedSizeBytes : 0;
+    if (bytes > max_dynamic) return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_dynamic)) !=
+        cudaSuccess)
+        return e;
+    raised.push_back({dev, func});
+    return cudaSuccess;
 }
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

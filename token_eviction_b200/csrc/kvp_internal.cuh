@@ -59,10 +59,11 @@ __host__ __device__ __forceinline__ int owner_of(long long t, long long T, long 
 }
 
 // Tiles by which a head-aligned cut's longest run may exceed the flat cut's and still be
-// chosen. Measured on the 32K layer (8 heads, 148 SMs), 15-tile head-aligned runs were
-// slower than 14-tile flat runs with one change of head, so the aligned cut is taken only
-// where it is no longer (short contexts, where a flat run would span many heads).
-constexpr int kHeadSwitchTiles = 0;
+// chosen. A run that changes head in mid-stream waits, at the start of its second head's
+// scoring pass, for that head's other runs and a fresh query block: on the 32K layer
+// (8 heads, 148 SMs) such runs ended about 16 us after the rest, while 15-tile aligned
+// runs ended within 3 us of each other.
+constexpr int kHeadSwitchTiles = 3;
 
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_score(const kvp_shape& s, const Plan& p, const uint16_t* q, const uint16_t* k,
@@ -74,6 +75,11 @@ cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t
                            const int32_t* idx, uint16_t* k_out, uint16_t* v_out, cudaStream_t st);
 
 int num_sms();
+
+// Lets `func` use up to `bytes` of dynamic shared memory on the current device. The limit
+// is per-device state: it is raised once per device and kernel (to the opt-in maximum
+// less the kernel's static shared memory), not on every call.
+cudaError_t allow_dynamic_smem(const void* func, size_t bytes);
 
 #ifdef KVP_CHECKS
 // Debug builds only: the first failed device-side bounds check (code, a, b) is recorded

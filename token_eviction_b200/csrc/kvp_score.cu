@@ -145,9 +145,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Rendezvous of all epilogue threads on an mbarrier, so that a thread that gives up a
-// wait can never leave the others blocked in a hardware barrier.
+// wait can never leave the others blocked in a hardware barrier. One arrival per warp,
+// after the warp's shared-memory writes are ordered before it.
 __device__ __forceinline__ bool epi_sync(SmemBars* sb, uint32_t& phase, int* err) {
-    ptx::mbar_arrive(&sb->epi);
+    __threadfence_block();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&sb->epi);
     const bool ok = wait_phase(&sb->epi, phase, sb, err, kErrWaitEpi);
     phase ^= 1u;
     return ok;
@@ -225,10 +228,12 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32]) {
     return v[0];
 }
 
-// Rare paths of the epilogue (tiles holding window keys, a ragged last chunk, logits
-// overflowing their row's offset) live in non-inlined functions that take only scalars
-// and load their chunk from TMEM themselves, so that the steady-state loops stay small
-// (the instruction cache holds them) and carry none of the rare paths' registers.
+// The one rare path of the epilogue (phase 0: logits far above their row's offset) is an
+// out-of-line function that takes only scalars and loads its chunk from TMEM itself, so
+// that the steady-state loops stay small (the instruction cache holds them) and carry
+// none of its registers. Masks (window keys, a ragged last chunk) stay in the steady-state
+// loops behind a warp-uniform flag: a separate masked path made the tile holding a head's
+// window keys the last of the whole launch to finish.
 
 // 32 TMEM columns of this warp's lanes at taddr: v[e] is the thread's key against local
 // column cbase + e, masked to -inf past the group's ncols columns and, inside the window
@@ -283,28 +288,14 @@ __device__ __noinline__ float2 lse_chunk_slow(uint32_t taddr, int cbase, int nco
     return make_float2(sum, lsum);
 }
 
-// Phase 0 hot path, one full chunk already in v (overwritten): lane L gets the warp's sum
-// of 2^(t - cw) for row L of the chunk; +inf or NaN tells the caller to take the rare path.
-__device__ __forceinline__ float lse_chunk_fast(float (&v)[32], const float* cw, float scale2) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-        const float4 c4 = *(const float4*)(cw + i);
-        v[i + 0] = ptx::ex2(fmaf(v[i + 0], scale2, -c4.x));
-        v[i + 1] = ptx::ex2(fmaf(v[i + 1], scale2, -c4.y));
-        v[i + 2] = ptx::ex2(fmaf(v[i + 2], scale2, -c4.z));
-        v[i + 3] = ptx::ex2(fmaf(v[i + 3], scale2, -c4.w));
-    }
-    return warp_reduce_scatter32<false>(v);
-}
-
-// Phase 0 hot path, two full chunks at once (offsets cw[0..63]): each element becomes
+// Phase 0 hot path, two chunks at once (row offsets cwx, cwy): each element becomes
 // 2^(t - cw) in place, the two chunks interleaved for independent work in flight.
-__device__ __forceinline__ void lse_pair_fast(float (&x)[32], float (&y)[32], const float* cw,
-                                              float scale2) {
+__device__ __forceinline__ void lse_pair_fast(float (&x)[32], float (&y)[32], const float* cwx,
+                                              const float* cwy, float scale2) {
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {
-        const float4 c4 = *(const float4*)(cw + i);
-        const float4 d4 = *(const float4*)(cw + 32 + i);
+        const float4 c4 = *(const float4*)(cwx + i);
+        const float4 d4 = *(const float4*)(cwy + i);
         x[i + 0] = ptx::ex2(fmaf(x[i + 0], scale2, -c4.x));
         x[i + 1] = ptx::ex2(fmaf(x[i + 1], scale2, -c4.y));
         x[i + 2] = ptx::ex2(fmaf(x[i + 2], scale2, -c4.z));
@@ -329,20 +320,23 @@ __device__ __forceinline__ void s1_chunk_fast(const float (&v)[32], const float*
     }
 }
 
-// Phase 1 rare path, one chunk loaded and masked here: the chunk's part of the key's S1.
-__device__ __noinline__ float s1_chunk_slow(uint32_t taddr, int cbase, int ncols, int col0, int jw,
-                                            const uint16_t* wpos, const float* lse2, float scale2) {
-    float v[32];
-    load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
-    float a0 = 0.f, a1 = 0.f;
+// Phase 1, one chunk with masks: columns from `nrem` on (past the group's last) and, for a
+// window key (jw > 0), query rows before the key contribute nothing.
+__device__ __forceinline__ void s1_chunk_masked(const float (&v)[32], const float* lse2, const uint16_t* wp,
+                                                int jw, int nrem, float scale2, float& a0, float& a1,
+                                                float& a2, float& a3) {
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        // masked entries (past the group's columns, or not visible) contribute nothing
-        const int n = col0 + cbase + e;
-        if (v[e] != -INFINITY) a0 += ptx::ex2(fmaf(v[e], scale2, -lse2[n]));
-        if (v[e + 1] != -INFINITY) a1 += ptx::ex2(fmaf(v[e + 1], scale2, -lse2[n + 1]));
+    for (int e = 0; e < 32; e += 4) {
+        const float4 l4 = *(const float4*)(lse2 + e);
+        const bool m0 = e + 0 < nrem && jw <= (int)wp[e + 0];
+        const bool m1 = e + 1 < nrem && jw <= (int)wp[e + 1];
+        const bool m2 = e + 2 < nrem && jw <= (int)wp[e + 2];
+        const bool m3 = e + 3 < nrem && jw <= (int)wp[e + 3];
+        a0 += m0 ? ptx::ex2(fmaf(v[e + 0], scale2, -l4.x)) : 0.f;
+        a1 += m1 ? ptx::ex2(fmaf(v[e + 1], scale2, -l4.y)) : 0.f;
+        a2 += m2 ? ptx::ex2(fmaf(v[e + 2], scale2, -l4.z)) : 0.f;
+        a3 += m3 ? ptx::ex2(fmaf(v[e + 3], scale2, -l4.w)) : 0.f;
     }
-    return a0 + a1;
 }
 
 }  // namespace
@@ -397,7 +391,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         ptx::mbar_init(&sb->qfull, 1);
         ptx::mbar_init(&sb->qempty, 1);
         ptx::mbar_init(&sb->fin, 1);
-        ptx::mbar_init(&sb->epi, kEpiThreads);
+        ptx::mbar_init(&sb->epi, kEpiThreads / 32);
         sb->abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -616,6 +610,10 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     const int j = key0 + lrow;                       // this thread's key
                     const int jw = j - window0;                      // > 0 only inside the window
                     // masks, needed only by warps holding window keys and by a ragged last chunk
+                    // masks: window keys (query rows before the key) and columns past the
+                    // group's last; only warps holding window keys or a ragged last chunk
+                    // need them, which the warp decides as a whole
+                    const bool masked = __any_sync(0xffffffffu, jw > 0) || (ncols & 31);
                     auto mask_chunk = [&](float (&v)[32], int c) {
                         if (jw > 0) {
 #pragma unroll
@@ -628,122 +626,76 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                                 if (c * 32 + e >= ncols) v[e] = -INFINITY;
                         }
                     };
-                    auto chunk0 = [&](float (&v)[32], int c) {
-                        mask_chunk(v, c);
-                        if (first_tile) {
-                            // offsets of the head's first tile: the logits of the warp's first
-                            // key (any offset within ~100 of a row's maximum keeps every
-                            // exponential finite; farther ones are caught below)
-                            __syncwarp();
-                            if (lane == 0) {
+                    // A head's first tile takes each row's offset from the warp's first key
+                    // (any offset within ~100 of a row's maximum keeps every exponential
+                    // finite; farther ones are caught by the overflow path).
+                    auto set_offsets = [&](const float (&v)[32], int c) {
+                        if (lane == 0) {
 #pragma unroll
-                                for (int e = 0; e < 32; ++e)
-                                    cwp[c * 32 + e] = v[e] == -INFINITY ? -1e30f : v[e] * p.scale2;
-                            }
-                            __syncwarp();
+                            for (int e = 0; e < 32; ++e)
+                                cwp[c * 32 + e] = v[e] == -INFINITY ? -1e30f : v[e] * p.scale2;
                         }
-                        float sum = lse_chunk_fast(v, cwp + c * 32, p.scale2);
-                        float lcur = 0.f;              // lane L: running sum of column c*32+L
-#pragma unroll
-                        for (int cc = 0; cc < 8; ++cc)
-                            if (cc == c) lcur = lw[cc];
-                        if (__any_sync(0xffffffffu, !(sum < INFINITY))) {
-                            // rare: a logit far above its row's offset; raise offsets, redo
-                            const float2 r = lse_chunk_slow(tstage + c * 32, c * 32, ncols, col0,
-                                                            jw, false, cwp + c * 32, wpos,
-                                                            p.scale2, lcur);
-                            sum = r.x;
-                            lcur = r.y;
-                        }
-                        lcur += sum;
-#pragma unroll
-                        for (int cc = 0; cc < 8; ++cc)
-                            if (cc == c) lw[cc] = lcur;
                     };
+                    // Two chunks at a time so that their exponentials and shuffles interleave;
+                    // an odd last chunk is paired with an empty one.
                     float x[32], y[32];
-                    // the path is chosen per warp: TMEM loads are warp-collective
-                    if (__any_sync(0xffffffffu, jw > 0) || (ncols & 31) || (nch & 1)) {
-                        // window keys, a ragged last chunk or an odd chunk count: masked,
-                        // chunk by chunk
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tstage, x);
-                        ptx::tmem_ld_wait(x);
-                        for (int c = 0; c < nch; c += 2) {
-                            const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
-                            if (has1) {
-                                __syncwarp();
-                                ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
-                            }
-                            chunk0(x, c);
-                            if (has1) {
-                                ptx::tmem_ld_wait(y);
-                                if (has2) {
-                                    __syncwarp();
-                                    ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
-                                }
-                                chunk0(y, c + 1);
-                                if (has2) ptx::tmem_ld_wait(x);
-                            }
-                        }
-                    } else {
-                        // steady state: whole chunks, no masks; two chunks at a time so that
-                        // their exponentials and shuffles interleave. A head's first tile
-                        // takes its row offsets from the warp's first key on the way.
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tstage, x);
-                        ptx::tmem_ld_wait(x);
+                    __syncwarp();
+                    ptx::tmem_ld_32x32b_x32(tstage, x);
+                    ptx::tmem_ld_wait(x);
 #pragma unroll 1
-                        for (int c = 0; c < nch; c += 2) {
+                    for (int c = 0; c < nch; c += 2) {
+                        const bool pair = c + 1 < nch;
+                        if (pair) {
                             __syncwarp();
                             ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
                             ptx::tmem_ld_wait(y);
-                            if (first_tile) {
-                                __syncwarp();
-                                if (lane == 0) {
+                        } else {
 #pragma unroll
-                                    for (int e = 0; e < 32; e += 4) {
-                                        *(float4*)(cwp + c * 32 + e) =
-                                            make_float4(x[e] * p.scale2, x[e + 1] * p.scale2,
-                                                        x[e + 2] * p.scale2, x[e + 3] * p.scale2);
-                                        *(float4*)(cwp + c * 32 + 32 + e) =
-                                            make_float4(y[e] * p.scale2, y[e + 1] * p.scale2,
-                                                        y[e + 2] * p.scale2, y[e + 3] * p.scale2);
-                                    }
-                                }
-                                __syncwarp();
+                            for (int e = 0; e < 32; ++e) y[e] = -INFINITY;
+                        }
+                        if (masked) {
+                            mask_chunk(x, c);
+                            if (pair) mask_chunk(y, c + 1);
+                        }
+                        if (first_tile) {
+                            __syncwarp();
+                            set_offsets(x, c);
+                            if (pair) set_offsets(y, c + 1);
+                            __syncwarp();
+                        }
+                        lse_pair_fast(x, y, cwp + c * 32, pair ? cwp + c * 32 + 32 : cwp + c * 32, p.scale2);
+                        float s0 = warp_reduce_scatter32<false>(x);
+                        float s1 = warp_reduce_scatter32<false>(y);
+                        float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+                        for (int cc = 0; cc < 8; cc += 2)
+                            if (cc == c) {
+                                l0 = lw[cc];
+                                l1 = lw[cc + 1];
                             }
-                            lse_pair_fast(x, y, cwp + c * 32, p.scale2);
-                            float s0 = warp_reduce_scatter32<false>(x);
-                            float s1 = warp_reduce_scatter32<false>(y);
-                            float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-                            for (int cc = 0; cc < 8; cc += 2)
-                                if (cc == c) {
-                                    l0 = lw[cc];
-                                    l1 = lw[cc + 1];
-                                }
-                            if (__any_sync(0xffffffffu, !(s0 < INFINITY) || !(s1 < INFINITY))) {
-                                // rare: a logit far above its row's offset; raise, redo
-                                float2 r = lse_chunk_slow(tstage + c * 32, c * 32, ncols, col0, jw, false,
-                                                          cwp + c * 32, wpos, p.scale2, l0);
-                                s0 = r.x;
-                                l0 = r.y;
-                                r = lse_chunk_slow(tstage + (c + 1) * 32, (c + 1) * 32, ncols, col0, jw, false,
-                                                   cwp + (c + 1) * 32, wpos, p.scale2, l1);
+                        if (__any_sync(0xffffffffu, !(s0 < INFINITY) || !(s1 < INFINITY))) {
+                            // rare: a logit far above its row's offset; raise, redo
+                            float2 r = lse_chunk_slow(tstage + c * 32, c * 32, ncols, col0, jw, false,
+                                                      cwp + c * 32, wpos, p.scale2, l0);
+                            s0 = r.x;
+                            l0 = r.y;
+                            if (pair) {
+                                r = lse_chunk_slow(tstage + (c + 1) * 32, (c + 1) * 32, ncols, col0, jw,
+                                                   false, cwp + (c + 1) * 32, wpos, p.scale2, l1);
                                 s1 = r.x;
                                 l1 = r.y;
                             }
+                        }
 #pragma unroll
-                            for (int cc = 0; cc < 8; cc += 2)
-                                if (cc == c) {
-                                    lw[cc] = l0 + s0;
-                                    lw[cc + 1] = l1 + s1;
-                                }
-                            if (c + 2 < nch) {
-                                __syncwarp();
-                                ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
-                                ptx::tmem_ld_wait(x);
+                        for (int cc = 0; cc < 8; cc += 2)
+                            if (cc == c) {
+                                lw[cc] = l0 + s0;
+                                if (pair) lw[cc + 1] = l1 + s1;
                             }
+                        if (c + 2 < nch) {
+                            __syncwarp();
+                            ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
+                            ptx::tmem_ld_wait(x);
                         }
                     }
                     first_tile = false;
@@ -835,31 +787,30 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 }
                 const int r0 = group_row0(head);
                 const int nslots = touch * kSlotsPerCta;
-                // Two threads per row, each folding every other slot with independent
-                // loads (online max/sum), then one exchange with the partner lane.
+                // Two threads per row, each over every other slot: first the row's
+                // maximum, then the sum of l 2^(m - max); every load and term independent.
                 for (int base = 0; base < 2 * p.rows; base += kEpiThreads) {
                     const int r2 = base + et, r = r2 >> 1;
-                    float M = -INFINITY, S = 0.f;
+                    const float2* pr = p.part + (size_t)(r0 + (r < p.rows ? r : 0)) * p.maxslots;
+                    float M = -INFINITY;
                     if (r < p.rows) {
-                        const float2* pr = p.part + (size_t)(r0 + r) * p.maxslots;
 #pragma unroll 4
                         for (int sl = r2 & 1; sl < nslots; sl += 2) {
                             const float2 ml = __ldcg(pr + sl);
-                            if (ml.x == -INFINITY || ml.y == 0.f) continue;
-                            if (ml.x > M) {
-                                S = S * ptx::ex2(M - ml.x) + ml.y;
-                                M = ml.x;
-                            } else {
-                                S += ml.y * ptx::ex2(ml.x - M);
-                            }
+                            if (ml.y != 0.f) M = fmaxf(M, ml.x);
                         }
                     }
-                    const float Mo = __shfl_xor_sync(0xffffffffu, M, 1);
-                    const float So = __shfl_xor_sync(0xffffffffu, S, 1);
-                    const float Mt = fmaxf(M, Mo);
-                    const float St = (M == -INFINITY ? 0.f : S * ptx::ex2(M - Mt)) +
-                                     (Mo == -INFINITY ? 0.f : So * ptx::ex2(Mo - Mt));
-                    if (r < p.rows && (r2 & 1) == 0) lse2[r] = Mt + __log2f(St);
+                    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+                    float S = 0.f;
+                    if (r < p.rows && M != -INFINITY) {
+#pragma unroll 4
+                        for (int sl = r2 & 1; sl < nslots; sl += 2) {
+                            const float2 ml = __ldcg(pr + sl);
+                            if (ml.y != 0.f) S += ml.y * ptx::ex2(ml.x - M);
+                        }
+                    }
+                    S += __shfl_xor_sync(0xffffffffu, S, 1);
+                    if (r < p.rows && (r2 & 1) == 0) lse2[r] = M + __log2f(S);
                 }
                 if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
                 for (long long t = a; t < b && ok; ++t, ++ait, ++pt) {
@@ -901,33 +852,35 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     const int col0 = (p.split && wg == 1) ? p.n1 : 0;        // first query row
                     const int ncols = p.split ? (wg == 0 ? p.n1 : p.rows - p.n1) : p.rows;
                     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                    // the path is chosen per warp: TMEM loads are warp-collective
-                    if (__any_sync(0xffffffffu, jw > 0) || (ncols & 31)) {
-                        // window keys or a ragged last chunk: masked, chunk by chunk
-                        for (int c = 0; c < nch; ++c)
-                            a0 += s1_chunk_slow(tstage + c * 32, c * 32, ncols, col0, jw, wpos, lse2,
-                                                p.scale2);
-                    } else {
-                        float x[32], y[32];
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tstage, x);
-                        ptx::tmem_ld_wait(x);
-                        for (int c = 0; c < nch; c += 2) {
-                            const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
-                            if (has1) {
+                    // masks (window keys, a ragged last chunk) are decided per warp: TMEM loads
+                    // are warp-collective, so every lane takes the same loop
+                    const bool masked = __any_sync(0xffffffffu, jw > 0) || (ncols & 31);
+                    auto s1_chunk = [&](const float (&v)[32], int c) {
+                        if (masked)
+                            s1_chunk_masked(v, lse2 + col0 + c * 32, wpos + col0 + c * 32, jw, ncols - c * 32,
+                                            p.scale2, a0, a1, a2, a3);
+                        else
+                            s1_chunk_fast(v, lse2 + col0 + c * 32, p.scale2, a0, a1, a2, a3);
+                    };
+                    float x[32], y[32];
+                    __syncwarp();
+                    ptx::tmem_ld_32x32b_x32(tstage, x);
+                    ptx::tmem_ld_wait(x);
+                    for (int c = 0; c < nch; c += 2) {
+                        const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
+                        if (has1) {
+                            __syncwarp();
+                            ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
+                        }
+                        s1_chunk(x, c);
+                        if (has1) {
+                            ptx::tmem_ld_wait(y);
+                            if (has2) {
                                 __syncwarp();
-                                ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
+                                ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
                             }
-                            s1_chunk_fast(x, lse2 + col0 + c * 32, p.scale2, a0, a1, a2, a3);
-                            if (has1) {
-                                ptx::tmem_ld_wait(y);
-                                if (has2) {
-                                    __syncwarp();
-                                    ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
-                                }
-                                s1_chunk_fast(y, lse2 + col0 + (c + 1) * 32, p.scale2, a0, a1, a2, a3);
-                                if (has2) ptx::tmem_ld_wait(x);
-                            }
+                            s1_chunk(y, c + 1);
+                            if (has2) ptx::tmem_ld_wait(x);
                         }
                     }
                     ptx::tc_fence_before();
@@ -1150,9 +1103,7 @@ cudaError_t launch_score(const kvp_shape& s, const Plan& plan, const uint16_t* q
 
     void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const Params) =
         D == 128 ? score_fused_tc<128> : score_fused_tc<64>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lc.smem)) !=
-        cudaSuccess)
-        return e;
+    if ((e = allow_dynamic_smem((const void*)kern, Lc.smem)) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(Lc.grid);
     cfg.blockDim = dim3(kThreads);

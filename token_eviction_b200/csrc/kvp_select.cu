@@ -252,9 +252,7 @@ cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score,
     cfg.numAttrs = 1;
     cudaError_t e;
     if (in_smem) {
-        e = cudaFuncSetAttribute(select_cluster<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)dyn);
-        if (e != cudaSuccess) return e;
+        if ((e = allow_dynamic_smem((const void*)select_cluster<true>, dyn)) != cudaSuccess) return e;
         return cudaLaunchKernelEx(&cfg, select_cluster<true>, score, idx, s.seq_len, s.window,
                                   s.budget, slice);
     }
