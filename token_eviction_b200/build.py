@@ -12,6 +12,7 @@ from __future__ import annotations
 
 import glob
 import os
+import re
 import subprocess
 import sys
 
@@ -29,6 +30,23 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--use_fast_math", "-Xcompiler", "-fP
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+
+# Translation units whose kernels must not spill registers. The scoring kernel issues
+# asynchronous TMEM loads (tcgen05.ld) and reads their registers only after
+# tcgen05.wait::ld; a spill or a reload of such a register in between would read or
+# clobber a register the load is still writing, so any spill there fails the build.
+NO_SPILL = ("kvp_score.cu",)
+
+
+def _check_no_spills(src: str, ptxas_log: str) -> None:
+    spills = re.findall(r"(\d+) bytes spill stores, (\d+) bytes spill loads", ptxas_log)
+    if not spills:
+        raise RuntimeError(f"{os.path.basename(src)}: no ptxas resource report to check")
+    bad = [(a, b) for a, b in spills if int(a) or int(b)]
+    if bad:
+        raise RuntimeError(f"{os.path.basename(src)}: register spills {bad}; its kernels must not "
+                           f"spill (asynchronous TMEM loads write registers in flight)")
 
 
 def _stale() -> bool:
@@ -52,10 +70,18 @@ def build(force: bool = False, verbose: bool = False, out: str | None = None,
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [NVCC, *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-c", src, "-o", obj]
-        if verbose:
+        checked = os.path.basename(src) in NO_SPILL
+        if verbose or checked:
             cmd.insert(1, "-Xptxas=-v")
+        if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.check_call(cmd)
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if verbose or res.returncode:
+            sys.stderr.write(res.stdout + res.stderr)
+        if res.returncode:
+            raise subprocess.CalledProcessError(res.returncode, cmd)
+        if checked:
+            _check_no_spills(src, res.stdout + res.stderr)
         objs.append(obj)
     tmp = target + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs])
