@@ -111,14 +111,14 @@ select_cluster(const float* __restrict__ score, int32_t* __restrict__ idx, int L
     uint32_t prefix = 0, mask = 0, krem = (uint32_t)kk;
     const int shifts[3] = {21, 10, 0};
     const uint32_t widths[3] = {2047u, 2047u, 1023u};
+    for (int b = tid; b < kBins; b += kSelThreads) {
+        sh.hist[b] = 0;
+        if (rank == 0) sh.merged[b] = 0;
+    }
+    cluster.sync();                        // histograms cleared (and keys staged)
     for (int pass = 0; pass < 3; ++pass) {
         const int shift = shifts[pass];
         const uint32_t dmask = widths[pass];
-        for (int b = tid; b < kBins; b += kSelThreads) {
-            sh.hist[b] = 0;
-            if (rank == 0) sh.merged[b] = 0;
-        }
-        cluster.sync();                    // merged histogram cleared (and keys staged)
         for (int j = lo + tid; j < hi; j += kSelThreads) {
             const uint32_t u = key_at(j);
             if ((u & mask) == prefix) atomicAdd(&sh.hist[(u >> shift) & dmask], 1u);
@@ -139,8 +139,13 @@ select_cluster(const float* __restrict__ score, int32_t* __restrict__ idx, int L
                 sh.digit = (unsigned)bl;
                 sh.krem = krem - above - ch;
             }
+            // every read of the merged histogram precedes the scan's barriers: clear it
+            // for the next pass under the same cluster barrier that publishes the digit
+            sh.merged[bh] = 0;
+            sh.merged[bl] = 0;
         }
-        cluster.sync();                    // digit published
+        for (int b = tid; b < kBins; b += kSelThreads) sh.hist[b] = 0;   // read above, by this thread
+        cluster.sync();                    // digit published, histograms cleared
         const unsigned dg = leader->digit, kr = leader->krem;
         prefix |= dg << shift;
         mask |= dmask << shift;
