@@ -89,3 +89,20 @@ def test_binding_validates_tensors_before_calling():
     cpu = torch.zeros((1, 4, 16, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         m.kvp_score(sh, cpu, cpu, cpu, cpu)
+
+
+def test_static_scratch_call_rejects_bad_arguments_on_the_host():
+    """kvp_score_static checks its arguments, and that the shape's scratch fits the
+    library's fixed array, before it touches the device."""
+    import token_eviction_b200 as m
+    f = m._lib.kvp_score_static
+    f.argtypes = [ctypes.c_void_p] * 8
+    f.restype = ctypes.c_int
+    ok = m.make_shape(1, 32, 8, 128, 4096, 32, 256)
+    assert f(ctypes.addressof(ok), None, 16, 16, 16, None, None, None) == 1          # NULL q_win
+    bad = m.make_shape(1, 32, 8, 100, 4096, 32, 256)
+    assert f(ctypes.addressof(bad), 16, 16, 16, 16, None, None, None) == 2          # d = 100
+    assert f(ctypes.addressof(ok), 16, 24, 16, 16, None, None, None) == 3           # misaligned k
+    big = m.make_shape(256, 32, 8, 128, 4096, 128, 256)
+    assert m.kvp_workspace_bytes(big) > (2 << 20)
+    assert f(ctypes.addressof(big), 16, 16, 16, 16, None, None, None) == 4          # over 2 MiB
