@@ -13,7 +13,11 @@ head mapping, a transposed operand, a wrong tie rule) fails at least one of them
   and the log-sum-exp with scipy;
 * planted |V| values give Eq. 4 exactly;
 * selection against numpy's stable lexsort, compaction against numpy indexing;
-* brute force with math.fsum on tiny inputs.
+* brute force with math.fsum on tiny inputs;
+* adding one vector to every key shifts each query row's logits by a constant and
+  leaves S1 unchanged (a softmax over the wrong axis fails this);
+* permuting the positions before the window permutes S1, S2 and S with them (a causal
+  bound measured from the wrong origin fails this).
 
 All run on the CPU (no GPU mark).
 """
@@ -240,3 +244,37 @@ def test_bad_shapes_raise():
         oracle.oracle_select(np.zeros((1, 10)), 3, 11)     # B > L
     with pytest.raises(ValueError):
         oracle.oracle_compact(k, v, np.array([[[0, 10]]], dtype=np.int32))
+
+
+def test_adding_one_vector_to_every_key_leaves_s1_unchanged():
+    # q . (k + u) = q . k + q . u shifts every logit of a query row by the same amount,
+    # so each softmax row, and S1, is unchanged. Small integers keep K and K + u exact
+    # in bf16, so the logits are exact in double on both sides.
+    b, hq, hkv, d, L, w = 1, 6, 3, 32, 40, 5
+    rng = np.random.default_rng(31)
+    q = bf16(rng.integers(-2, 3, (b, hq, w, d)) / 4.0)
+    k = rng.integers(-3, 4, (b, hkv, L, d)).astype(np.float64)
+    u = rng.integers(-3, 4, (1, hkv, 1, d)).astype(np.float64)
+    v = bf16(rng.standard_normal((b, hkv, L, d)))
+    s1a, s2a, _ = oracle.oracle_score(q, bf16(k), v)
+    s1b, s2b, _ = oracle.oracle_score(q, bf16(k + u), v)
+    np.testing.assert_allclose(s1b, s1a, rtol=1e-10)
+    np.testing.assert_array_equal(s2b, s2a)
+
+
+def test_permuting_keys_before_the_window_permutes_the_scores():
+    # Every window query sees every position before the window, so moving a (K, V) row
+    # there moves its S1, S2 and S with it; window positions stay put.
+    b, hq, hkv, d, L, w = 2, 4, 2, 16, 37, 6
+    q, k, v = rand_inputs(b, hq, hkv, d, L, w, seed=41)
+    n = L - w
+    perm = np.random.default_rng(42).permutation(n)
+    kp, vp = k.copy(), v.copy()
+    kp[:, :, :n] = k[:, :, perm]
+    vp[:, :, :n] = v[:, :, perm]
+    s1, s2, s = oracle.oracle_score(q, k, v)
+    s1p, s2p, sp = oracle.oracle_score(q, kp, vp)
+    np.testing.assert_allclose(s1p[..., :n], s1[..., perm], rtol=1e-10)
+    np.testing.assert_array_equal(s2p[..., :n], s2[..., perm])
+    np.testing.assert_allclose(sp[..., :n], s[..., perm], rtol=1e-10)
+    np.testing.assert_allclose(s1p[..., n:], s1[..., n:], rtol=1e-10)
