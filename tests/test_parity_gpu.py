@@ -72,6 +72,11 @@ SMALL = {
     # more than 256 query rows per KV head: accumulators split across two TMEM stages
     "split_ragged_g5": synth.small("llama8b_32k", hq=10, hkv=2, seq_len=900, window=56, budget=150),
     "split_wide_window": synth.small("tiny", hq=2, hkv=2, head_dim=128, seq_len=700, window=300, budget=400),
+    # one 256-column accumulator stage per epilogue group (128 < G w <= 256)
+    "wide_stage_g8": synth.small("llama8b_32k", hq=8, hkv=1, seq_len=1100, window=32, budget=200),
+    "wide_stage_g7": synth.small("llama8b_32k", hq=14, hkv=2, seq_len=777, window=32, budget=150),
+    # d = 64 with every tile split across both groups (G w > 256)
+    "split_d64": synth.small("tiny", hq=6, hkv=1, seq_len=900, window=48, budget=200),
 }
 
 
