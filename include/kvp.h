@@ -22,9 +22,10 @@
  *   - All tensors are device memory, contiguous, row-major, innermost dimension last.
  *     bf16 tensors are passed as their 16-bit patterns (uint16_t).
  *   - Query head hq belongs to KV head hq / G, G = hq_count / hkv_count.
- *   - The caller owns and allocates every buffer. The library allocates no device
- *     memory and keeps no state between calls; calls with distinct workspaces may run
- *     concurrently from several host threads.
+ *   - The caller owns and allocates every buffer. No call allocates device memory
+ *     (kvp_score_static uses a fixed array that the library defines instead of a
+ *     workspace) and no call keeps data for the next; calls with distinct workspaces
+ *     may run concurrently from several host threads.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls only enqueue
  *     work and never synchronise the host.
  *   - Argument errors are detected on the host before anything is launched; the outputs
