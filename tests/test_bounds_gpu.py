@@ -42,11 +42,21 @@ class Arena:
         assert bad.size == 0, f"{bad.size} canary words overwritten, first at byte {bad[0] * 4}"
 
 
+# shapes beyond the named workloads: one 256-column TMEM stage per group, split tiles at
+# d = 64, and long head-aligned runs
+EXTRA = {
+    "wide_stage_g8": synth.small("llama8b_32k", hq=8, hkv=1, seq_len=1100, window=32, budget=200),
+    "split_d64": synth.small("tiny", hq=6, hkv=1, seq_len=900, window=48, budget=200),
+    "long_128k_b10": synth.WORKLOADS["long_128k_b10"],
+}
+
+
 @pytest.mark.parametrize("name,budget", [("tiny", None), ("llama8b_32k", None), ("llama8b_32k", 128),
-                                         ("gqa7_batched", None)])
+                                         ("gqa7_batched", None), ("wide_stage_g8", None),
+                                         ("split_d64", None), ("long_128k_b10", None)])
 def test_no_write_outside_buffers(name, budget):
     import token_eviction_b200 as m
-    wl = synth.WORKLOADS[name]
+    wl = EXTRA.get(name) or synth.WORKLOADS[name]
     B = wl.budget if budget is None else budget
     b, hq, hkv, d, L, w = wl.batch, wl.hq, wl.hkv, wl.head_dim, wl.seq_len, wl.window
     sh = m.make_shape(b, hq, hkv, d, L, w, B)
