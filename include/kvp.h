@@ -30,8 +30,11 @@
  *     work and never synchronise the host.
  *   - Argument errors are detected on the host before anything is launched; the outputs
  *     are then untouched. A launch failure returns KVP_ERR_CUDA; kvp_last_cuda_error()
- *     names the CUDA error. Every device-side wait is bounded in time, so no kernel can
- *     hang.
+ *     names the CUDA error.
+ *   - Every device-side wait is bounded in time, so no kernel can hang. A wait that gives
+ *     up records an error code in the workspace and its kernel returns early: the call
+ *     has already returned KVP_OK, and its outputs are undefined. kvp_workspace_status()
+ *     reads that code back.
  */
 #ifndef KVP_H_
 #define KVP_H_
@@ -67,7 +70,7 @@ typedef enum {
     KVP_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned */
     KVP_ERR_WORKSPACE = 4, /* workspace NULL or smaller than kvp_workspace_bytes() */
     KVP_ERR_CUDA = 5,      /* a CUDA runtime/driver call or kernel launch failed */
-    KVP_ERR_TIMEOUT = 6    /* reserved: a bounded device-side wait gave up */
+    KVP_ERR_TIMEOUT = 6    /* a bounded device-side wait gave up (see kvp_workspace_status) */
 } kvp_status;
 
 /* Bytes of device workspace that kvp_score and kvp_select need for `shape`
@@ -110,6 +113,18 @@ KVP_API kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const 
                                const int32_t* idx, uint16_t* k_out, uint16_t* v_out, void* stream);
 
 /*
+ * Device-side status of the last kvp_score call that used `workspace`: KVP_ERR_TIMEOUT if
+ * one of its bounded waits gave up (the call's score, s1 and s2 are then undefined, and so
+ * is whatever kvp_select and kvp_compact made from them), KVP_OK otherwise. The code sits in
+ * the workspace's first 4 bytes; kvp_score clears it when it starts.
+ *   workspace  the device workspace passed to kvp_score (16-byte aligned)
+ *   stream     the stream kvp_score ran on
+ * This call synchronises `stream` (it copies the 4 bytes to the host), so it cannot be
+ * made during stream capture: it then returns KVP_ERR_CUDA. NULL workspace: KVP_ERR_NULL.
+ */
+KVP_API kvp_status kvp_workspace_status(const void* workspace, void* stream);
+
+/*
  * kvp_score without a workspace, for callers that cannot allocate device memory at the
  * time they evict: a serving engine that reserved the device for its own memory pool at
  * start-up, code that may not allocate after initialisation, or a runtime that only
@@ -121,8 +136,9 @@ KVP_API kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const 
  * that loads the library holds it until the process exits. A shape whose
  * kvp_workspace_bytes() exceeds KVP_STATIC_SCRATCH_BYTES is rejected with
  * KVP_ERR_WORKSPACE before anything is launched.
- *   - The first call on each device looks up the array's device address (once per
- *     device); make that first call before any stream capture on that device.
+ *   - Every call looks up the array's device address with cudaGetSymbolAddress, which
+ *     allocates nothing; the first lookup on a device may load the library's device code
+ *     there, so make the first call on each device before any stream capture.
  *   - All calls share the one array: calls that may overlap on the GPU (other streams,
  *     other host threads, concurrent graphs) race and must be serialised by the caller.
  *     Each call clears the parts of the array that must start at zero.
@@ -133,6 +149,10 @@ KVP_API kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const 
 KVP_API kvp_status kvp_score_static(const kvp_shape* shape, const uint16_t* q_win,
                                     const uint16_t* k, const uint16_t* v, float* score,
                                     float* s1, float* s2, void* stream);
+
+/* kvp_workspace_status for kvp_score_static: the device-side status of the last call on
+ * this device, read from the library's scratch array (synchronises `stream`). */
+KVP_API kvp_status kvp_score_static_status(void* stream);
 
 /* The name of the CUDA error behind the calling thread's most recent KVP_ERR_CUDA
  * ("cudaSuccess" if there was none). Host-only; never fails. */

@@ -19,8 +19,14 @@ def declared_symbols():
 
 
 def test_header_declares_the_boundary():
-    assert {"kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact",
-            "kvp_status_string"} <= declared_symbols()
+    assert {"kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact", "kvp_workspace_status",
+            "kvp_score_static", "kvp_score_static_status", "kvp_status_string",
+            "kvp_last_cuda_error"} <= declared_symbols()
+
+
+def test_binding_lists_every_declared_symbol():
+    import token_eviction_b200 as m
+    assert declared_symbols() == set(m.EXPORTED)
 
 
 def test_library_exports_every_declared_symbol():
@@ -106,3 +112,23 @@ def test_static_scratch_call_rejects_bad_arguments_on_the_host():
     big = m.make_shape(256, 32, 8, 128, 4096, 128, 256)
     assert m.kvp_workspace_bytes(big) > (2 << 20)
     assert f(ctypes.addressof(big), 16, 16, 16, 16, None, None, None) == 4          # over 2 MiB
+
+
+def test_status_call_rejects_bad_workspace_on_the_host():
+    import token_eviction_b200 as m
+    assert m._lib.kvp_workspace_status(None, None) == 1      # KVP_ERR_NULL
+    assert m._lib.kvp_workspace_status(24, None) == 3        # KVP_ERR_ALIGN
+
+
+def test_static_call_names_the_cuda_error_behind_a_failure():
+    """Without a device, kvp_score_static fails when it looks up its scratch array; the
+    CUDA error must then be the one kvp_last_cuda_error() names."""
+    import torch
+    import token_eviction_b200 as m
+    if torch.cuda.is_available():
+        pytest.skip("needs a host without a usable CUDA device")
+    ok = m.make_shape(1, 32, 8, 128, 4096, 32, 256)
+    st = m._lib.kvp_score_static(ctypes.byref(ok), 16, 16, 16, 16, None, None, None)
+    assert st == 5                                            # KVP_ERR_CUDA
+    assert m.kvp_last_cuda_error() != "cudaSuccess"
+    assert m._lib.kvp_score_static_status(None) == 5

@@ -29,8 +29,9 @@ def _lib():
     return m, f
 
 
-@pytest.mark.parametrize("name", ["llama8b_32k", "gqa7_batched", "tiny"])
-def test_static_scratch_matches_workspace_call(name):
+@pytest.mark.parametrize("name,with_s1_s2", [("llama8b_32k", True), ("gqa7_batched", True), ("tiny", True),
+                                             ("long_128k_b10", False), ("llama8b_32k", False)])
+def test_static_scratch_matches_workspace_call(name, with_s1_s2):
     m, kvp_score_static = _lib()
     wl = synth.WORKLOADS[name]
     inp = synth.make_inputs(wl)
@@ -41,12 +42,14 @@ def test_static_scratch_matches_workspace_call(name):
     ref = [torch.empty((b, hkv, L), dtype=torch.float32, device="cuda") for _ in range(3)]
     m.kvp_score(sh, q, k, v, *ref)
     stream = torch.cuda.current_stream().cuda_stream
+    nout = 3 if with_s1_s2 else 1
     for _ in range(2):                     # two calls in a row reuse the same scratch
         out = [torch.full((b, hkv, L), float("nan"), dtype=torch.float32, device="cuda")
-               for _ in range(3)]
-        st = kvp_score_static(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                              out[0].data_ptr(), out[1].data_ptr(), out[2].data_ptr(), stream)
+               for _ in range(nout)]
+        ptrs = [t.data_ptr() for t in out] + [None] * (3 - nout)
+        st = kvp_score_static(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(), *ptrs, stream)
         assert st == 0, m.kvp_status_string(st)
+        assert m._lib.kvp_score_static_status(stream) == 0
         torch.cuda.synchronize()
         for got, want, what in zip(out, ref, ("S", "S1", "S2")):
             check_scores(got.cpu().numpy(), want.cpu().numpy().astype(np.float64), what)

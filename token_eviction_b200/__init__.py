@@ -11,6 +11,7 @@ The functions carry the C names:
 * ``kvp_score(shape, q_win, k, v, score, s1=None, s2=None, workspace=None, stream=None)``
 * ``kvp_select(shape, score, idx, workspace=None, stream=None)``
 * ``kvp_compact(shape, k, v, idx, k_out, v_out, stream=None)``
+* ``kvp_workspace_status(workspace, stream=None)``
 * ``kvp_status_string(status)``
 
 plus ``evict_layer``, which allocates the outputs and runs all three calls.
@@ -74,6 +75,12 @@ def _load():
     lib.kvp_status_string.restype = ctypes.c_char_p
     lib.kvp_last_cuda_error.argtypes = []
     lib.kvp_last_cuda_error.restype = ctypes.c_char_p
+    lib.kvp_workspace_status.argtypes = [P, P]
+    lib.kvp_workspace_status.restype = ctypes.c_int
+    lib.kvp_score_static.argtypes = [S, P, P, P, P, P, P, P]
+    lib.kvp_score_static.restype = ctypes.c_int
+    lib.kvp_score_static_status.argtypes = [P]
+    lib.kvp_score_static_status.restype = ctypes.c_int
     return lib
 
 
@@ -84,8 +91,8 @@ _lib = _load()
 # enqueues one small memset of its workspace counters.
 KERNELS_PER_LAYER = 3
 
-EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact", "kvp_status_string",
-            "kvp_last_cuda_error")
+EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact", "kvp_workspace_status",
+            "kvp_score_static", "kvp_score_static_status", "kvp_status_string", "kvp_last_cuda_error")
 
 
 def make_shape(batch, hq, hkv, head_dim, seq_len, window, budget) -> KvpShape:
@@ -159,6 +166,14 @@ def kvp_score(shape, q_win, k, v, score, s1=None, s2=None, workspace=None, strea
                         _stream(stream))
     if st != KVP_OK:
         raise KvpError(st, "kvp_score")
+
+
+def kvp_workspace_status(workspace, stream=None) -> int:
+    """Device-side status of the last kvp_score on `workspace`: KVP_OK (0) or
+    KVP_ERR_TIMEOUT (6) when one of its bounded waits gave up. Synchronises the stream."""
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    return int(_lib.kvp_workspace_status(workspace.data_ptr(), _stream(stream)))
 
 
 def kvp_select(shape, score, idx, workspace=None, stream=None):

@@ -89,6 +89,23 @@ def build(force: bool = False, verbose: bool = False, out: str | None = None,
     return target
 
 
+# The debug build: device-side bounds checks that record the first failure instead of
+# touching memory out of bounds, and the fault-injection hook the tests use to make a
+# bounded wait run out (kvp_debug_set_fault).
+CHECKS_LIB = os.path.join(PKG, "libkvp_checks.so")
+
+
+def build_checks(force: bool = False, verbose: bool = False) -> str:
+    if not force and os.path.exists(CHECKS_LIB):
+        t = os.path.getmtime(CHECKS_LIB)
+        deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+        if all(os.path.getmtime(f) <= t for f in deps):
+            return CHECKS_LIB
+    return build(force=True, verbose=verbose, out=CHECKS_LIB, defines=("KVP_CHECKS",))
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="-v" in sys.argv)
     print(LIB)
+    if "--checks" in sys.argv:
+        print(build_checks(force="--force" in sys.argv, verbose="-v" in sys.argv))

@@ -87,11 +87,12 @@ bool plan_of(const kvp_shape& s, Plan* p) {
                                     owner_of(f, T, p->grid, tph, p->cph) + 1);
     }
     p->maxslots = slots * kSlotsPerCta;
+    // the error word sits at offset 0 of every workspace, so that a status read needs no shape
     size_t off = 0;
-    p->off_done = off;
-    off += align_up((size_t)units * sizeof(uint32_t), 256);
     p->off_err = off;
     off += 256;
+    p->off_done = off;
+    off += align_up((size_t)units * sizeof(uint32_t), 256);
     p->off_part = off;
     off += align_up((size_t)s.batch * s.hq * s.window * p->maxslots * sizeof(float2), 256);
     p->off_select = off;
@@ -109,11 +110,25 @@ static bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 // The CUDA error behind the calling thread's last KVP_ERR_CUDA (cudaSuccess if none).
 static thread_local cudaError_t t_last_cuda_error = cudaSuccess;
 
-static kvp_status cuda_failed(cudaError_t e) {
+namespace kvp {
+
+kvp_status record_cuda_error(cudaError_t e) {
     t_last_cuda_error = e;
     cudaGetLastError();  // clear the runtime's sticky copy of a launch error
     return KVP_ERR_CUDA;
 }
+
+kvp_status read_error_word(const void* workspace, cudaStream_t stream) {
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    return word != 0 ? KVP_ERR_TIMEOUT : KVP_OK;
+}
+
+}  // namespace kvp
+
+static kvp_status cuda_failed(cudaError_t e) { return record_cuda_error(e); }
 
 extern "C" size_t kvp_workspace_bytes(const kvp_shape* shape) {
     Plan p;
@@ -166,7 +181,19 @@ extern "C" kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, con
     return KVP_OK;
 }
 
+extern "C" kvp_status kvp_workspace_status(const void* workspace, void* stream) {
+    if (!workspace) return KVP_ERR_NULL;
+    if (!aligned16(workspace)) return KVP_ERR_ALIGN;
+    return read_error_word(workspace, (cudaStream_t)stream);
+}
+
 #ifdef KVP_CHECKS
+// Debug builds only: every later scoring call waits for `extra_peers` completions per head
+// that never come, and gives up any device wait after `wait_limit_ns` (0: the default).
+extern "C" KVP_API void kvp_debug_set_fault(int extra_peers, unsigned long long wait_limit_ns) {
+    set_fault(extra_peers, wait_limit_ns);
+}
+
 // Debug builds only: copy out (and clear) the first failed device-side bounds check.
 extern "C" KVP_API int kvp_debug_take_check_unit(int unit, int* out4) {
     int (*readers[3])(int*) = {take_check_score, take_check_select, take_check_compact};

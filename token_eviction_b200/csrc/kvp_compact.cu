@@ -1,10 +1,11 @@
-// Compaction of the K/V cache to the kept positions: a 16-byte vectorised row gather.
+// Compaction of the K/V cache to the kept positions: a vectorised row gather.
 //
 // k_out[b, h, t, :] = k[b, h, idx[b, h, t], :] and the same for v, as a bit copy (the
 // eviction step of "Preserving Large Activations: The Key to KV Cache Pruning",
-// Listing 1: the cache keeps max_capacity_prompt positions). Each thread moves one
-// 16-byte piece of one kept K row and the same piece of the V row; a grid of
-// whole waves over the SMs strides over all pieces.
+// Listing 1: the cache keeps max_capacity_prompt positions). Each thread moves four
+// consecutive 16-byte pieces of one kept K row and the same pieces of the V row, with all
+// eight loads issued before any store so that enough bytes are in flight to keep HBM busy;
+// a grid of whole waves over the SMs strides over all pieces.
 #include <cuda_runtime.h>
 
 #include "kvp_internal.cuh"
@@ -12,28 +13,39 @@
 namespace kvp {
 namespace {
 
-__global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ k,
-                                                   const uint4* __restrict__ v,
-                                                   const int32_t* __restrict__ idx,
-                                                   uint4* __restrict__ k_out,
-                                                   uint4* __restrict__ v_out, int L, int B,
-                                                   int piece_shift, int total, int rows_total) {
+constexpr int kPiecesPerThread = 4;   // 16-byte pieces of K (and of V) per thread
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads) gather_rows(const uint4* __restrict__ k,
+                                                        const uint4* __restrict__ v,
+                                                        const int32_t* __restrict__ idx,
+                                                        uint4* __restrict__ k_out,
+                                                        uint4* __restrict__ v_out, int L, int B,
+                                                        int piece_shift, int items, int rows_total) {
     const int stride = gridDim.x * blockDim.x;
     const int pmask = (1 << piece_shift) - 1;
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+    for (int it = blockIdx.x * blockDim.x + threadIdx.x; it < items; it += stride) {
+        const int e = it * kPiecesPerThread;  // first piece (row pieces are a multiple of 4)
         const int rt = e >> piece_shift;      // (row, t): which kept row
         const int c = e & pmask;              // which 16-byte piece of it
         const int row = rt / B;
         const int j = __ldg(idx + rt);
-        uint4 a = make_uint4(0, 0, 0, 0), b = a;
+        uint4 a[kPiecesPerThread], b[kPiecesPerThread];
         if (j >= 0 && j < L) {
             const size_t src = (((size_t)row * L + j) << piece_shift) + c;
-            a = __ldg(k + src);
-            b = __ldg(v + src);
+#pragma unroll
+            for (int q = 0; q < kPiecesPerThread; ++q) a[q] = __ldg(k + src + q);
+#pragma unroll
+            for (int q = 0; q < kPiecesPerThread; ++q) b[q] = __ldg(v + src + q);
+        } else {
+#pragma unroll
+            for (int q = 0; q < kPiecesPerThread; ++q) a[q] = b[q] = make_uint4(0, 0, 0, 0);
         }
         if (!KVP_CHECK(row < rows_total, 301, row, rt)) continue;
-        __stcs(k_out + e, a);
-        __stcs(v_out + e, b);
+#pragma unroll
+        for (int q = 0; q < kPiecesPerThread; ++q) __stcs(k_out + e + q, a[q]);
+#pragma unroll
+        for (int q = 0; q < kPiecesPerThread; ++q) __stcs(v_out + e + q, b[q]);
     }
 }
 
@@ -44,14 +56,18 @@ cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t
     const int piece_shift = s.head_dim == 128 ? 4 : 3;  // 16-byte pieces per row: 16 or 8
     const long long total = ((long long)s.batch * s.hkv * s.budget) << piece_shift;
     if (total > INT32_MAX) return cudaErrorInvalidValue;
-    const long long want = (total + 255) / 256;
-    const int sms = num_sms();
-    const long long cap = (long long)sms * 8;  // 8 resident CTAs of 256 threads per SM
-    const int grid = (int)(want < cap ? want : cap);
-    gather_rows<<<grid, 256, 0, st>>>((const uint4*)k, (const uint4*)v, idx, (uint4*)k_out,
-                                      (uint4*)v_out, s.seq_len, s.budget, piece_shift, (int)total,
-                                      s.batch * s.hkv);
-    return cudaGetLastError();
+    const long long items = total / kPiecesPerThread;
+    const long long want = (items + kThreads - 1) / kThreads;
+    const long long cap = (long long)num_sms() * 8;  // 8 resident CTAs of 256 threads per SM
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(want < cap ? want : cap));
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = st;
+    // launched with cudaLaunchKernelEx: its return value is this launch's own error, never
+    // a sticky error left by an earlier, unrelated launch
+    return cudaLaunchKernelEx(&cfg, gather_rows, (const uint4*)k, (const uint4*)v, idx, (uint4*)k_out,
+                              (uint4*)v_out, s.seq_len, s.budget, piece_shift, (int)items,
+                              s.batch * s.hkv);
 }
 
 #ifdef KVP_CHECKS

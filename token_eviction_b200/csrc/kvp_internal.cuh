@@ -26,8 +26,8 @@ struct Plan {
     int grid;            // CTAs of the scoring kernel (one per SM, at most one per tile)
     int cph;             // runs per KV head when runs are head-aligned; 0: flat runs
     int maxslots;        // partial-softmax slots per query row (CTAs touching one head)
+    size_t off_err;      // int: first device-side error code (0 = none); always offset 0
     size_t off_done;     // uint32 per (sequence, KV head): CTAs done with phase 0
-    size_t off_err;      // int: first device-side error code (0 = none)
     size_t off_part;     // float2 (max, sum) partials [b*hq*w][maxslots], log2 domain
     size_t off_select;   // selection scratch
     size_t bytes;        // total workspace
@@ -76,6 +76,14 @@ cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t
 
 int num_sms();
 
+// Records `e` as the calling thread's last CUDA error (what kvp_last_cuda_error() names),
+// clears the runtime's sticky copy of a launch error, and returns KVP_ERR_CUDA.
+kvp_status record_cuda_error(cudaError_t e);
+
+// Reads the error word at the start of a workspace (synchronising `stream`): KVP_OK,
+// KVP_ERR_TIMEOUT when a bounded device wait gave up, or KVP_ERR_CUDA.
+kvp_status read_error_word(const void* workspace, cudaStream_t stream);
+
 // Lets `func` use up to `bytes` of dynamic shared memory on the current device. The limit
 // is per-device state: it is raised once per device and kernel (to the opt-in maximum
 // less the kernel's static shared memory), not on every call.
@@ -93,9 +101,10 @@ static __device__ int g_kvp_check[4];
         return cudaMemcpyToSymbol(g_kvp_check, zero, sizeof(zero)) == cudaSuccess ? 0 : -1; \
     }
 int take_check_score(int* out4);
+void set_fault(int extra_peers, unsigned long long wait_limit_ns);
 int take_check_select(int* out4);
 int take_check_compact(int* out4);
-__device__ __forceinline__ void kvp_check_fail(int code, int a, int b) {
+static __device__ __noinline__ void kvp_check_fail(int code, int a, int b) {
     if (atomicCAS(&g_kvp_check[0], 0, code) == 0) {
         g_kvp_check[1] = a;
         g_kvp_check[2] = b;

@@ -7,30 +7,29 @@
 //   Eq. 5  S[j]  = S1[j] * S2[j]
 // Window query i sits at position L - w + i and sees keys j <= L - w + i.
 //
-// The softmax denominators must be known before any key's S1 can be summed, so K is
-// swept twice; both sweeps run inside one kernel. In both, tcgen05 computes the tile's
-// logits transposed, D[key, row] = K_tile[key] . Q_group[row] (M = 128 keys, N = G w
-// query rows), so every epilogue thread owns one key and each TMEM column is a query row.
-//   phase 0 (log-sum-exp): each CTA owns a contiguous run of 128-key tiles of the
-//     flattened (sequence, KV head, tile) space. Per query row, each warp keeps a running
-//     offset and sum of 2^(t - offset) over its 32 keys, t = logit * log2(e) / sqrt(d);
-//     a butterfly reduce-scatter turns a 32 x 32 chunk of exponentials into per-row sums.
-//     At the end of each KV head in its run, a CTA combines its warps' (offset, sum)
-//     pairs, publishes one slot per row and bumps the head's completion counter.
-//   phase 1 (scores): the same CTA sweeps the same tiles again (K now mostly from L2).
-//     Before its first tile of a head it waits (bounded) until every CTA touching that
-//     head has published, then merges the slots into lse2 = M + log2(sum_s l_s 2^(m_s - M))
-//     per row. Per tile each thread sums 2^(t - lse2) over its key's row columns, reads
-//     the key's V row once from shared memory for S2, and writes S (and S1, S2 if asked).
-// Loads go through a ring of tile slots in shared memory: phase 0 streams K through all
-// of them; phase 1 gives V (from HBM) the larger share and K (mostly L2) the rest.
-// Warp roles: warp 0 issues TMA loads (the ring and the group's query rows), warp 1
-// allocates TMEM and issues the MMAs from one thread, and two epilogue warpgroups
-// (warps 2-5 and 6-9, one TMEM lane quarter per warp) each own TMEM accumulator
-// stages. When a tile's accumulator fits one stage (G w <= 256) the groups take
-// alternate tiles; otherwise every tile is split across both stages (query-row halves in
-// phase 0, column halves in phase 1) and the second group hands its partial S1 to the
-// first through shared memory.
+// A softmax row's denominator must be known before any key's S1 can be summed, so K is
+// swept twice; both sweeps run inside one kernel. Each CTA owns a contiguous run of
+// 128-key tiles of the flattened (sequence, KV head, tile) space.
+//   phase 0 (log-sum-exp; one query row per thread): tcgen05 computes
+//     D[row, key] = Q_group[row] . K_tile[key]  (M = 128 rows of one row block, N = keys),
+//     so each epilogue thread owns one query row (a TMEM lane) and keeps its running
+//     offset m and sum l = sum_j 2^(t_j - m) in registers, t = logit * log2(e) / sqrt(d).
+//     At the end of each KV head in its run a CTA publishes one (m, l) slot per row to
+//     the workspace and bumps the head's completion counter.
+//   phase 1 (scores; one key per thread): the same tiles again (K now mostly from L2),
+//     with D[key, row] = K_tile[key] . Q_group[row]  (M = 128 keys, N = query rows).
+//     Before its first tile of a head a CTA waits (bounded) until every CTA touching the
+//     head has published, then merges the slots into lse2 = M + log2(sum_s l_s 2^(m_s-M))
+//     per row. Per tile each thread sums 2^(t - lse2) over its key's query rows: S1.
+//   S2 is reduced from each V tile, staged once in shared memory, by two warps of its own,
+//   so that V's arrival from HBM never stalls the exponentials.
+// Warp roles: warp 0 issues TMA loads (a ring of tile slots and the group's query rows),
+// warp 1 allocates TMEM and issues the MMAs from one thread, warps 2-3 reduce V tiles to
+// S2, and two epilogue warpgroups (warps 4-7 and 8-11, one TMEM lane quarter per warp)
+// read the accumulators. TMEM holds four accumulator stages of 128 columns; a tile's work
+// is cut into units of at most 128 columns (phase 0: a run of keys over every row block;
+// phase 1: a part of the query rows), unit k takes stage k % 4, and stage s belongs to
+// epilogue group s % 2.
 // Every wait is bounded by a timer; a wait that gives up records an error code in the
 // workspace and the CTA unwinds without touching TMEM or shared memory still in use.
 #include <cuda.h>
@@ -50,68 +49,70 @@ namespace kvp {
 namespace {
 
 constexpr int kTile = 128;                        // keys per tile
-constexpr int kEpiGroups = 2;                     // epilogue warpgroups
-constexpr int kEpiThreads = 128 * kEpiGroups;
-constexpr int kThreads = 64 + kEpiThreads;        // + TMA warp + MMA warp
-constexpr int kMaxSlots = 8;                     // tile slots of the load ring
-constexpr size_t kRingBytes = 128 * 1024;        // at most this much of it in flight (see build_launch)
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kMaxStageCols = 256;           // widest accumulator stage
+constexpr int kGroups = 2;                        // epilogue warpgroups
+constexpr int kStages = 4;                        // TMEM accumulator stages
+constexpr int kStageCols = 128;                   // TMEM columns per stage
+constexpr uint32_t kTmemCols = kStages * kStageCols;
+constexpr int kWarpS2 = 2, kS2Warps = 2;          // warps that reduce V tiles to S2
+constexpr int kWarpEpi = kWarpS2 + kS2Warps;      // first epilogue warp
+constexpr int kEpiThreads = 128 * kGroups;
+constexpr int kThreads = 32 * kWarpEpi + kEpiThreads;
+constexpr int kMaxSlots = 8;                      // tile slots of the load ring
+constexpr int kS2Bufs = 4;                        // S2 hand-off buffers (one tile each)
+constexpr int kCombBufs = 2;                      // partial-S1 hand-off buffers
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s on any single wait
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMinSmem = 116 * 1024;              // forces one CTA per SM (TMEM is taken whole)
 constexpr int kQBoxRows = 64;
-constexpr size_t kBarBytes = 512;                 // shared memory reserved for SmemBars
+constexpr size_t kBarBytes = 640;                 // shared memory reserved for SmemBars
+constexpr float kSumLimit = 1.8446744e19f;        // 2^64: a chunk sum above it raises the offset
 
 #ifdef KVP_TRACE
 // Debug builds only: %globaltimer stamps per CTA at phase boundaries.
 __device__ unsigned long long g_kvp_trace[kPlanGrid][8];
 #define KVP_STAMP(i) (g_kvp_trace[blockIdx.x][(i)] = ptx::globaltimer_ns())
-// per-tile events of the first 4 CTAs: [cta][tile][event]
+// per-tile events of four CTAs: [cta][tile][event]
 __device__ unsigned long long g_kvp_ttrace[4][64][8];
-// MMA-thread steps of the first 4 CTAs (clock64): [cta][tile][step]
 __device__ long long g_kvp_mtrace[4][64][12];
-#define KVP_MSTAMP(t, e) ((blockIdx.x < 4 && (t) < 64) ? (void)(g_kvp_mtrace[blockIdx.x][(t)][(e)] = clock64()) : (void)0)
 __device__ __forceinline__ int kvp_trace_slot() {
-    return blockIdx.x == 0 ? 0 : blockIdx.x == 18 ? 1 : blockIdx.x == 73 ? 2 : blockIdx.x == 147 ? 3 : -1;
+    return blockIdx.x == 0 ? 0 : blockIdx.x == 18 ? 1 : blockIdx.x == 73 ? 2 : blockIdx.x == 143 ? 3 : -1;
 }
 #define KVP_TSTAMP(t, e) \
     ((kvp_trace_slot() >= 0 && (t) < 64) ? (void)(g_kvp_ttrace[kvp_trace_slot()][(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
 #else
 #define KVP_STAMP(i) ((void)0)
 #define KVP_TSTAMP(t, e) ((void)0)
-#define KVP_MSTAMP(t, e) ((void)0)
 #endif
 
 // error codes recorded in the workspace (first one wins)
-enum : int { kErrWaitTma = 1, kErrWaitMma = 2, kErrWaitEpi = 3, kErrWaitPeers = 4 };
+enum : int { kErrWaitTma = 1, kErrWaitMma = 2, kErrWaitEpi = 3, kErrWaitPeers = 4, kErrWaitS2 = 5 };
 
 struct Params {
-    int L, w, G, rows, hq, hkv, D;
-    int qrows;           // query rows staged in shared memory (rows rounded up to 64)
-    int n1, n2;          // phase 1 MMA N of the two column chunks (n2 = 0: one chunk)
-    int split;           // 0: groups alternate tiles; 1: every tile split over both stages
-    int stage_cols;      // TMEM columns per accumulator stage (128 or 256)
-    int spg;             // accumulator stages per epilogue group (2 when a stage is 128 wide)
+    int L, w, rows, hq, hkv, G;
+    int nrb, nk0, u0, lg_cpb;  // phase 0: row blocks, keys per unit, units per tile, log2(nk0 / 32)
+    int p1, n1, rows16;        // phase 1: parts per tile, rows per part, rows rounded up to 16
+    int qrows;                 // query rows staged in shared memory (rows rounded up to 64)
     int tiles_per_head, total_tiles, grid, cph, maxslots;
-    int ns, nk1, nv1;    // ring slots; phase 1 gives K slots [0, nk1), V slots [nk1, ns)
-    float scale2;        // log2(e) / sqrt(d)
-    uint32_t q_bytes, k_bytes, v_bytes;
-    uint32_t off_q, off_slots, off_lse, off_cw, off_wpos, off_bar;
-    int cw_stride;       // floats per epilogue warp of phase 0 row offsets
+    int ns, nk1, nv1;          // ring slots; phase 1 gives K slots [0, nk1), V slots [nk1, ns)
+    float scale2;              // log2(e) / sqrt(d)
+    uint32_t q_bytes, tile_bytes;
+    uint32_t off_slots, off_lse, off_comb, off_s2, off_stage, off_wpos, off_bar;
+    int extra_peers;           // fault injection (debug builds): peers that never arrive
+    unsigned long long wait_limit_ns;
     float* score;
     float* s1;
     float* s2;
-    float2* part;        // [b*hq*w][maxslots]: (max, sum) in log2 units
-    uint32_t* done;      // [b*hkv]
+    float2* part;              // [b*hq*w][maxslots]: (max, sum) in log2 units
+    uint32_t* done;            // [b*hkv]
     int* err;
 };
 
 struct SmemBars {
     uint64_t kfull[kMaxSlots], kempty[kMaxSlots];   // per slot, for its K loads
     uint64_t vfull[kMaxSlots], vempty[kMaxSlots];   // per phase 1 V slot (index s - nk1)
-    uint64_t accfull[4], accempty[4];
-    uint64_t combfull[2], combempty[2];
+    uint64_t accfull[kStages], accempty[kStages];
+    uint64_t combfull[kCombBufs], combempty[kCombBufs];
+    uint64_t s2full[kS2Bufs], s2empty[kS2Bufs];
     uint64_t qfull, qempty, fin;
     uint64_t epi;        // rendezvous of all epilogue threads
     uint32_t tmem_base;
@@ -121,7 +122,7 @@ struct SmemBars {
 // Wait for phase `parity` of `bar`; false if the CTA is unwinding or the wait timed out
 // (then the first error code is recorded and the CTA told to unwind).
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemBars* sb,
-                                           int* err, int code) {
+                                           const Params& p, int code) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer_ns();
     while (true) {
@@ -129,8 +130,8 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemB
         for (int i = 0; i < 32; ++i)
             if (ptx::mbar_try_wait(bar, parity)) return true;
         if (*(volatile int*)&sb->abort_flag) return false;
-        if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-            atomicCAS(err, 0, code);
+        if (ptx::globaltimer_ns() - t0 > p.wait_limit_ns) {
+            atomicCAS(p.err, 0, code);
             *(volatile int*)&sb->abort_flag = 1;
             return false;
         }
@@ -138,7 +139,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemB
 }
 
 // Wait for phase `parity` of `bar` for at most the wait limit, whatever the CTA's state:
-// used before exit, so that no copy is still writing this CTA's shared memory.
+// used before exit, so that no copy or MMA is still writing this CTA's memory.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = ptx::globaltimer_ns();
     while (!ptx::mbar_try_wait(bar, parity))
@@ -147,12 +148,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 // Rendezvous of all epilogue threads on an mbarrier, so that a thread that gives up a
 // wait can never leave the others blocked in a hardware barrier. One arrival per warp,
-// after the warp's shared-memory writes are ordered before it.
-__device__ __forceinline__ bool epi_sync(SmemBars* sb, uint32_t& phase, int* err) {
+// after the warp's memory writes are ordered before it.
+__device__ __forceinline__ bool epi_sync(SmemBars* sb, uint32_t& phase, const Params& p) {
     __threadfence_block();
     __syncwarp();
     if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&sb->epi);
-    const bool ok = wait_phase(&sb->epi, phase, sb, err, kErrWaitEpi);
+    const bool ok = wait_phase(&sb->epi, phase, sb, p, kErrWaitEpi);
     phase ^= 1u;
     return ok;
 }
@@ -164,26 +165,30 @@ __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
     return *reinterpret_cast<uint32_t*>(&m);
 }
 
-// Accumulator stage that epilogue group g uses for the CTA's tile number i, and the
-// parity of that use. Alternate-tile mode: group i & 1 takes tile i, cycling through its
-// spg stages (stages g, g + 2); split mode: group g takes stage g of every tile.
-__device__ __forceinline__ int acc_stage(int split, int spg, int i, int g, uint32_t& parity) {
-    if (split) {
-        parity = (uint32_t)i & 1u;
-        return g;
+// max |v| over the D bf16 values of one row in shared memory, read in 16-byte pieces in a
+// rotated order per lane (consecutive lanes hit distinct bank groups).
+template <int D>
+__device__ __forceinline__ float row_absmax(const uint8_t* row, int lane) {
+    constexpr int kPieces = D * 2 / 16;
+    const uint4* r = reinterpret_cast<const uint4*>(row);
+    uint32_t mx = 0;
+#pragma unroll
+    for (int c = 0; c < kPieces; ++c) {
+        const uint4 x = r[(c + lane) & (kPieces - 1)];
+        mx = bf16x2_absmax(mx, x.x & 0x7FFF7FFFu);
+        mx = bf16x2_absmax(mx, x.y & 0x7FFF7FFFu);
+        mx = bf16x2_absmax(mx, x.z & 0x7FFF7FFFu);
+        mx = bf16x2_absmax(mx, x.w & 0x7FFF7FFFu);
     }
-    const int u = i >> 1;
-    parity = (uint32_t)(u / spg) & 1u;
-    return g + 2 * (u % spg);
+    return fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
 }
 
-// The load ring. Phase 0 streams only K, through all ns slots in turn; phase 1 streams K
-// through slots [0, nk1) and V through slots [nk1, ns). Each slot's K loads are counted
-// across both phases, so the parity of a slot's barriers follows from the tile number.
-__device__ __forceinline__ int ring_uses(int s, int period, int n) {   // uses of slot s
-    return n > s ? (n - s + period - 1) / period : 0;                   // among n tiles
+// Uses of ring position s among the first n uses of a ring of `period` positions.
+__device__ __forceinline__ int ring_uses(int s, int period, int n) {
+    return n > s ? (n - s + period - 1) / period : 0;
 }
 // K slot of the run's tile i in `phase`, and the number of that slot's earlier K loads.
+// Phase 0 streams K through all ns slots in turn; phase 1 through slots [0, nk1).
 __device__ __forceinline__ int k_slot(int phase, int i, int n, const Params& p, int& use) {
     if (phase == 0) {
         use = i / p.ns;
@@ -209,142 +214,89 @@ struct RunIter {
     }
 };
 
-// Butterfly reduce-scatter across the 32 lanes of a warp: v[i] holds this lane's value of
-// column i; on return lane L's v[0] holds the maximum (kMax) or sum over all 32 lanes of
-// column L. Five rounds, 31 shuffles.
-template <bool kMax>
-__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32]) {
-    const int lane = threadIdx.x & 31;
+// Element i of a 4-entry register array with a run-time index, without local memory.
+template <typename T>
+__device__ __forceinline__ T pick4(const T (&a)[4], int i) {
+    return i == 0 ? a[0] : i == 1 ? a[1] : i == 2 ? a[2] : a[3];
+}
+template <typename T>
+__device__ __forceinline__ void put4(T (&a)[4], int i, T x) {
+    a[0] = i == 0 ? x : a[0];
+    a[1] = i == 1 ? x : a[1];
+    a[2] = i == 2 ? x : a[2];
+    a[3] = i == 3 ? x : a[3];
+}
+
+// Phase 0, one chunk of 32 keys of one query row (v: raw logits, -inf where masked):
+// adds sum_e 2^(v_e * scale2 - m) to l. The offset m is raised (and l rescaled) only when
+// a chunk sum would exceed 2^64, which also covers the head's first chunk (m = -inf).
+__device__ __forceinline__ void lse_chunk(const float (&v)[32], float scale2, float& m, float& l) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-    for (int k = 16; k >= 1; k >>= 1) {
-        const bool upper = (lane & k) != 0;
+    for (int e = 0; e < 32; e += 4) {
+        a0 += ptx::ex2(fmaf(v[e + 0], scale2, -m));
+        a1 += ptx::ex2(fmaf(v[e + 1], scale2, -m));
+        a2 += ptx::ex2(fmaf(v[e + 2], scale2, -m));
+        a3 += ptx::ex2(fmaf(v[e + 3], scale2, -m));
+    }
+    float cs = (a0 + a1) + (a2 + a3);
+    if (__any_sync(0xffffffffu, !(cs <= kSumLimit))) {
+        // rare: the chunk holds logits far above this row's offset (or the offset is unset)
+        float mc = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < k; ++i) {
-            const float send = upper ? v[i] : v[i + k];
-            const float keep = upper ? v[i + k] : v[i];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, k);
-            v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+        for (int e = 0; e < 32; ++e) mc = fmaxf(mc, v[e]);
+        mc *= scale2;
+        if (mc > m) {
+            l *= ptx::ex2(m - mc);                 // m = -inf: l is 0 and stays 0
+            m = mc;
+        }
+        cs = 0.f;
+        if (m != -INFINITY) {
+            a0 = a1 = a2 = a3 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+                a0 += ptx::ex2(fmaf(v[e + 0], scale2, -m));
+                a1 += ptx::ex2(fmaf(v[e + 1], scale2, -m));
+                a2 += ptx::ex2(fmaf(v[e + 2], scale2, -m));
+                a3 += ptx::ex2(fmaf(v[e + 3], scale2, -m));
+            }
+            cs = (a0 + a1) + (a2 + a3);
         }
     }
-    return v[0];
+    l += cs;
 }
 
-// The one rare path of the epilogue (phase 0: logits far above their row's offset) is an
-// out-of-line function that takes only scalars and loads its chunk from TMEM itself, so
-// that the steady-state loops stay small (the instruction cache holds them) and carry
-// none of its registers. Masks (window keys, a ragged last chunk) stay in the steady-state
-// loops behind a warp-uniform flag: a separate masked path made the tile holding a head's
-// window keys the last of the whole launch to finish.
-
-// 32 TMEM columns of this warp's lanes at taddr: v[e] is the thread's key against local
-// column cbase + e, masked to -inf past the group's ncols columns and, inside the window
-// (key offset jw > 0), for query rows before the key.
-__device__ __forceinline__ void load_masked(uint32_t taddr, float (&v)[32], int cbase, int ncols,
-                                            int col0, int jw, const uint16_t* wpos) {
-    __syncwarp();
-    ptx::tmem_ld_32x32b_x32(taddr, v);
-    ptx::tmem_ld_wait(v);
+// Phase 1, one chunk of 32 query rows of one key: adds 2^(v_e * scale2 - lse2_e). With
+// `masked`, rows from `nrem` on (past the part's last) contribute nothing, nor, for a
+// window key (jw > 0), rows whose window position is before the key.
+__device__ __forceinline__ float s1_chunk(const float (&v)[32], const float* lse2, const uint16_t* wp,
+                                          bool masked, int jw, int nrem, float scale2) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    if (!masked) {
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const int n = cbase + e;
-        if (n >= ncols || (jw > 0 && jw > (int)wpos[col0 + n])) v[e] = -INFINITY;
+        for (int e = 0; e < 32; e += 4) {
+            const float4 l4 = *(const float4*)(lse2 + e);
+            a0 += ptx::ex2(fmaf(v[e + 0], scale2, -l4.x));
+            a1 += ptx::ex2(fmaf(v[e + 1], scale2, -l4.y));
+            a2 += ptx::ex2(fmaf(v[e + 2], scale2, -l4.z));
+            a3 += ptx::ex2(fmaf(v[e + 3], scale2, -l4.w));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+            const float4 l4 = *(const float4*)(lse2 + e);
+            const bool m0 = e + 0 < nrem && jw <= (int)wp[e + 0];
+            const bool m1 = e + 1 < nrem && jw <= (int)wp[e + 1];
+            const bool m2 = e + 2 < nrem && jw <= (int)wp[e + 2];
+            const bool m3 = e + 3 < nrem && jw <= (int)wp[e + 3];
+            a0 += m0 ? ptx::ex2(fmaf(v[e + 0], scale2, -l4.x)) : 0.f;
+            a1 += m1 ? ptx::ex2(fmaf(v[e + 1], scale2, -l4.y)) : 0.f;
+            a2 += m2 ? ptx::ex2(fmaf(v[e + 2], scale2, -l4.z)) : 0.f;
+            a3 += m3 ? ptx::ex2(fmaf(v[e + 3], scale2, -l4.w)) : 0.f;
+        }
     }
+    return (a0 + a1) + (a2 + a3);
 }
-
-// Phase 0, one chunk on the rare path. cw[0..31]: the warp's offsets (log2 units) of the
-// chunk's rows; `first` sets them to each row's maximum over the warp's keys. Returns
-// (lane L's sum of 2^(t - cw) over the warp's keys for row L of the chunk, lsum rescaled
-// if the offsets had to be raised to keep the exponentials finite).
-__device__ __noinline__ float2 lse_chunk_slow(uint32_t taddr, int cbase, int ncols, int col0,
-                                              int jw, bool first, float* cw,
-                                              const uint16_t* wpos, float scale2, float lsum) {
-    const int lane = threadIdx.x & 31;
-    float v[32];
-    load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
-    if (first) {
-        const float cmax = warp_reduce_scatter32<true>(v);
-        __syncwarp();
-        cw[lane] = cmax == -INFINITY ? -1e30f : cmax * scale2;
-        __syncwarp();
-        load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = ptx::ex2(fmaf(v[i], scale2, -cw[i]));
-    float sum = warp_reduce_scatter32<false>(v);
-    if (__any_sync(0xffffffffu, !(sum < INFINITY))) {
-        load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = fmaf(v[i], scale2, -cw[i]);
-        float d = warp_reduce_scatter32<true>(v);
-        d = d > 0.f ? d : 0.f;                    // also maps NaN (all masked) to 0
-        lsum *= ptx::ex2(-d);
-        __syncwarp();
-        cw[lane] += d;
-        __syncwarp();
-        load_masked(taddr, v, cbase, ncols, col0, jw, wpos);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = ptx::ex2(fmaf(v[i], scale2, -cw[i]));
-        sum = warp_reduce_scatter32<false>(v);
-    }
-    return make_float2(sum, lsum);
-}
-
-// Phase 0 hot path, two chunks at once (row offsets cwx, cwy): each element becomes
-// 2^(t - cw) in place, the two chunks interleaved for independent work in flight.
-__device__ __forceinline__ void lse_pair_fast(float (&x)[32], float (&y)[32], const float* cwx,
-                                              const float* cwy, float scale2) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-        const float4 c4 = *(const float4*)(cwx + i);
-        const float4 d4 = *(const float4*)(cwy + i);
-        x[i + 0] = ptx::ex2(fmaf(x[i + 0], scale2, -c4.x));
-        x[i + 1] = ptx::ex2(fmaf(x[i + 1], scale2, -c4.y));
-        x[i + 2] = ptx::ex2(fmaf(x[i + 2], scale2, -c4.z));
-        x[i + 3] = ptx::ex2(fmaf(x[i + 3], scale2, -c4.w));
-        y[i + 0] = ptx::ex2(fmaf(y[i + 0], scale2, -d4.x));
-        y[i + 1] = ptx::ex2(fmaf(y[i + 1], scale2, -d4.y));
-        y[i + 2] = ptx::ex2(fmaf(y[i + 2], scale2, -d4.z));
-        y[i + 3] = ptx::ex2(fmaf(y[i + 3], scale2, -d4.w));
-    }
-}
-
-// Phase 1 hot path, one full chunk: add 2^(t - lse2[n0 + e]) over its 32 query rows.
-__device__ __forceinline__ void s1_chunk_fast(const float (&v)[32], const float* lse2, float scale2,
-                                              float& a0, float& a1, float& a2, float& a3) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-        const float4 l4 = *(const float4*)(lse2 + e);
-        a0 += ptx::ex2(fmaf(v[e + 0], scale2, -l4.x));
-        a1 += ptx::ex2(fmaf(v[e + 1], scale2, -l4.y));
-        a2 += ptx::ex2(fmaf(v[e + 2], scale2, -l4.z));
-        a3 += ptx::ex2(fmaf(v[e + 3], scale2, -l4.w));
-    }
-}
-
-// Phase 1, one chunk with masks: columns from `nrem` on (past the group's last) and, for a
-// window key (jw > 0), query rows before the key contribute nothing.
-__device__ __forceinline__ void s1_chunk_masked(const float (&v)[32], const float* lse2, const uint16_t* wp,
-                                                int jw, int nrem, float scale2, float& a0, float& a1,
-                                                float& a2, float& a3) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-        const float4 l4 = *(const float4*)(lse2 + e);
-        const bool m0 = e + 0 < nrem && jw <= (int)wp[e + 0];
-        const bool m1 = e + 1 < nrem && jw <= (int)wp[e + 1];
-        const bool m2 = e + 2 < nrem && jw <= (int)wp[e + 2];
-        const bool m3 = e + 3 < nrem && jw <= (int)wp[e + 3];
-        a0 += m0 ? ptx::ex2(fmaf(v[e + 0], scale2, -l4.x)) : 0.f;
-        a1 += m1 ? ptx::ex2(fmaf(v[e + 1], scale2, -l4.y)) : 0.f;
-        a2 += m2 ? ptx::ex2(fmaf(v[e + 2], scale2, -l4.z)) : 0.f;
-        a3 += m3 ? ptx::ex2(fmaf(v[e + 3], scale2, -l4.w)) : 0.f;
-    }
-}
-
-}  // namespace
-}  // namespace kvp
-
-namespace kvp {
-namespace {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -352,15 +304,13 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                const __grid_constant__ CUtensorMap vmap, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t* Qs = smem + p.off_q;
-    uint8_t* Slots = smem + p.off_slots;               // ring slots of tile_bytes each
-    float* lse2 = (float*)(smem + p.off_lse);          // [rows, padded to 4]
-    float* comb = lse2 + ((p.rows + 3) & ~3);           // [2][128] partial S1 handoff (split mode)
-    // phase 0: [8 warps][cw_stride] row offsets; at the end of a head the same bytes stage
-    // the warps' (offset, sum) pairs as float2 [8][cw_stride]
-    float* cw_all = (float*)(smem + p.off_cw);
-    // window position i of query row n (row n = g * w + i), so no division in the loops
-    uint16_t* wpos = (uint16_t*)(smem + p.off_wpos);
+    uint8_t* Qs = smem;                                  // [D / 64][qrows][64] bf16, 128B swizzle
+    uint8_t* Slots = smem + p.off_slots;                 // ring slots of tile_bytes each
+    float* lse2 = (float*)(smem + p.off_lse);            // [rows, padded to 4]
+    float* comb = (float*)(smem + p.off_comb);           // [kCombBufs][128] partial S1 hand-off
+    float* s2buf = (float*)(smem + p.off_s2);            // [kS2Bufs][128] S2 of a tile's keys
+    float2* stage0 = (float2*)(smem + p.off_stage);      // [rows] phase 0 group hand-off
+    uint16_t* wpos = (uint16_t*)(smem + p.off_wpos);     // window position of query row n: n % w
     SmemBars* sb = (SmemBars*)(smem + p.off_bar);
 
     constexpr int kHalves = D / 64;                 // 128-byte swizzle rows per operand row
@@ -372,22 +322,28 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const long long T = p.total_tiles;
     const long long t0 = run_begin(blockIdx.x, T, p.grid, p.tiles_per_head, p.cph);
     const long long t1 = run_begin(blockIdx.x + 1, T, p.grid, p.tiles_per_head, p.cph);
+    const int n = (int)(t1 - t0);                   // tiles in this CTA's run
+    const int U0 = n * p.u0;                        // phase 0 units of the run
 
-    for (int n = threadIdx.x; n < p.rows; n += kThreads) wpos[n] = (uint16_t)(n % p.w);
+    for (int r = threadIdx.x; r < p.rows; r += kThreads) wpos[r] = (uint16_t)(r % p.w);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxSlots; ++s) {
             ptx::mbar_init(&sb->kfull[s], 1);
             ptx::mbar_init(&sb->kempty[s], 1);
             ptx::mbar_init(&sb->vfull[s], 1);
-            ptx::mbar_init(&sb->vempty[s], 4);
+            ptx::mbar_init(&sb->vempty[s], kS2Warps);
         }
-        for (int s = 0; s < 4; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(&sb->accfull[s], 1);
             ptx::mbar_init(&sb->accempty[s], 4);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kCombBufs; ++s) {
             ptx::mbar_init(&sb->combfull[s], 4);
             ptx::mbar_init(&sb->combempty[s], 4);
+        }
+        for (int s = 0; s < kS2Bufs; ++s) {
+            ptx::mbar_init(&sb->s2full[s], kS2Warps);
+            ptx::mbar_init(&sb->s2empty[s], 4);
         }
         ptx::mbar_init(&sb->qfull, 1);
         ptx::mbar_init(&sb->qempty, 1);
@@ -410,12 +366,6 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     ptx::tc_fence_after();
     const uint32_t tmem = sb->tmem_base;
     if (threadIdx.x == 0) KVP_STAMP(0);
-#ifdef KVP_TRACE
-    if (threadIdx.x == 0 && blockIdx.x < 4) {
-        g_kvp_ttrace[blockIdx.x][63][0] = clock64();
-        g_kvp_ttrace[blockIdx.x][63][1] = ptx::globaltimer_ns();
-    }
-#endif
 
     auto group_row0 = [&](int bh) {
         const int b = bh / p.hkv, h = bh % p.hkv;
@@ -425,11 +375,9 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // K is read again by phase 1; plain L2 eviction measured a little faster than
-            // marking it evict-last (K alone fits in L2 at 32K, K and V do not)
+            // K is read again by phase 1 (from L2 when it fits); V and phase 1's K stream
             const uint64_t pol_keep = ptx::policy_evict_normal();
             const uint64_t pol_stream = ptx::policy_evict_first();
-            const int n = (int)(t1 - t0);
             int qgen = 0, cur = -1;
             int kiss[kMaxSlots] = {}, viss[kMaxSlots] = {};   // loads issued per slot
             bool ok = true;
@@ -440,7 +388,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 int i = 0;                                  // tile number within the run
                 while (ok && it.next(head, a, b)) {
                     if (head != cur) {
-                        if (qgen > 0 && !(ok = wait_phase(&sb->qempty, (qgen - 1) & 1, sb, p.err, kErrWaitTma))) break;
+                        if (qgen > 0 && !(ok = wait_phase(&sb->qempty, (qgen - 1) & 1, sb, p, kErrWaitTma))) break;
                         ptx::mbar_arrive_expect_tx(&sb->qfull, p.q_bytes);
                         const int r0 = group_row0(head);
                         for (int rb = 0; rb < p.qrows; rb += kQBoxRows)
@@ -454,9 +402,9 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
                         int use;
                         const int s = k_slot(phase, i, n, p, use);
-                        if (!(ok = wait_phase(&sb->kempty[s], (use & 1) ^ 1, sb, p.err, kErrWaitTma))) break;
+                        if (!(ok = wait_phase(&sb->kempty[s], (use & 1) ^ 1, sb, p, kErrWaitTma))) break;
                         KVP_TSTAMP(phase * n + i, 0);
-                        ptx::mbar_arrive_expect_tx(&sb->kfull[s], p.k_bytes);
+                        ptx::mbar_arrive_expect_tx(&sb->kfull[s], p.tile_bytes);
                         for (int c = 0; c < kHalves; ++c)
                             ptx::tma_load_3d(Slots + s * kSlotBytes + c * kHalfTile, &kmap, &sb->kfull[s],
                                              c * 64, key0, head, phase == 0 ? pol_keep : pol_stream);
@@ -464,11 +412,11 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         if (phase == 1) {
                             const int jv = i % p.nv1, sv = p.nk1 + jv, vuse = i / p.nv1;
                             // a V slot's first load waits for its last K load of phase 0 to be consumed
-                            const int u0 = vuse == 0 ? ring_uses(sv, p.ns, n) : 0;
-                            if (u0 > 0 && !(ok = wait_phase(&sb->kempty[sv], (u0 - 1) & 1, sb, p.err, kErrWaitTma))) break;
-                            if (!(ok = wait_phase(&sb->vempty[jv], (vuse & 1) ^ 1, sb, p.err, kErrWaitTma))) break;
+                            const int u0s = vuse == 0 ? ring_uses(sv, p.ns, n) : 0;
+                            if (u0s > 0 && !(ok = wait_phase(&sb->kempty[sv], (u0s - 1) & 1, sb, p, kErrWaitTma))) break;
+                            if (!(ok = wait_phase(&sb->vempty[jv], (vuse & 1) ^ 1, sb, p, kErrWaitTma))) break;
                             KVP_TSTAMP(phase * n + i, 6);
-                            ptx::mbar_arrive_expect_tx(&sb->vfull[jv], p.v_bytes);
+                            ptx::mbar_arrive_expect_tx(&sb->vfull[jv], p.tile_bytes);
                             ptx::tma_load_3d(Slots + sv * kSlotBytes, &vmap, &sb->vfull[jv], 0, key0, head,
                                              pol_stream);
                             ++viss[jv];
@@ -479,8 +427,8 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             }
             // Never leave with copies in flight: wait for the last load issued to every slot
             // (these waits do not stop early when the CTA unwinds).
-            for (int s2 = 0; s2 < p.ns; ++s2)
-                if (kiss[s2] > 0) drain_wait(&sb->kfull[s2], (kiss[s2] - 1) & 1);
+            for (int s = 0; s < p.ns; ++s)
+                if (kiss[s] > 0) drain_wait(&sb->kfull[s], (kiss[s] - 1) & 1);
             for (int jv = 0; jv < p.nv1; ++jv)
                 if (viss[jv] > 0) drain_wait(&sb->vfull[jv], (viss[jv] - 1) & 1);
             if (qgen > 0) drain_wait(&sb->qfull, (qgen - 1) & 1);
@@ -488,74 +436,69 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc1a = ptx::idesc_bf16_f32(128, p.n1);
-            const uint32_t idesc1b = ptx::idesc_bf16_f32(128, p.n2 > 0 ? p.n2 : 16);
             const uint32_t q_addr = ptx::smem_u32(Qs), k_addr = ptx::smem_u32(Slots);
-            const int n = (int)(t1 - t0);
-            int ait = 0, qgen = 0, cur = -1;
+            const uint32_t idesc0 = ptx::idesc_bf16_f32(128, p.nk0);
+            int qgen = 0, cur = -1;
             bool ok = true;
             for (int phase = 0; phase < 2 && ok; ++phase) {
                 RunIter it(t0, t1, p.tiles_per_head);
                 int head;
                 long long a, b;
                 int i = 0;                                  // tile number within the run
+                int unit = 0;                               // unit number within the phase
                 while (ok && it.next(head, a, b)) {
                     if (head != cur) {
-                        if (!(ok = wait_phase(&sb->qfull, qgen & 1, sb, p.err, kErrWaitMma))) break;
+                        if (!(ok = wait_phase(&sb->qfull, qgen & 1, sb, p, kErrWaitMma))) break;
                         ++qgen;
                         cur = head;
                         ptx::tc_fence_after();
                     }
-                    for (long long t = a; t < b; ++t, ++i) {
-                        const int kit = phase * n + i;              // trace index
-                        (void)kit;
-                        int use;
-                        const int s = k_slot(phase, i, n, p, use);
-                        if (!(ok = wait_phase(&sb->kfull[s], use & 1, sb, p.err, kErrWaitMma))) break;
-                        KVP_TSTAMP(kit, 1);
-                        KVP_MSTAMP(kit, 0);
+                    for (long long t = a; t < b && ok; ++t, ++i) {
+                        int kuse;
+                        const int s = k_slot(phase, i, n, p, kuse);
+                        if (!(ok = wait_phase(&sb->kfull[s], kuse & 1, sb, p, kErrWaitMma))) break;
+                        KVP_TSTAMP(phase * n + i, 1);
                         const uint32_t kbase = k_addr + s * kSlotBytes;
-                        // stages written for this tile: one (alternating) or both (split)
-                        const int g_lo = p.split ? 0 : (ait & 1);
-                        const int g_hi = p.split ? 1 : (ait & 1);
-                        for (int g = g_lo; g <= g_hi && ok; ++g) {
-                            uint32_t use_parity;
-                            const int st = acc_stage(p.split, p.spg, ait, g, use_parity);
-                            if (!(ok = wait_phase(&sb->accempty[st], use_parity ^ 1, sb, p.err, kErrWaitMma))) break;
-                            KVP_TSTAMP(kit, 2);
-                            KVP_MSTAMP(kit, 1);
+                        const int nunits = phase == 0 ? p.u0 : p.p1;
+                        for (int j = 0; j < nunits; ++j, ++unit) {
+                            const int st = unit & (kStages - 1);
+                            const int use = (phase == 0 ? 0 : ring_uses(st, kStages, U0)) + unit / kStages;
+                            if (!(ok = wait_phase(&sb->accempty[st], (use & 1) ^ 1, sb, p, kErrWaitMma))) break;
                             ptx::tc_fence_after();
-                            KVP_MSTAMP(kit, 2);
-                            const uint32_t d0 = tmem + (uint32_t)(st * p.stage_cols);
-                            // descriptors of the first k-step; later k-steps add byte
-                            // offsets (in 16-byte units) to the start-address field
-                            const uint64_t kdesc0 = ptx::sw128_kmajor_desc(kbase);
-                            const uint64_t qdesc0 = ptx::sw128_kmajor_desc(q_addr);
-                            const bool first_chunk = !p.split || g == 0;
-                            const bool second_chunk = p.n2 > 0 && (!p.split || g == 1);
-                            const uint32_t n2_col = p.split ? 0u : (uint32_t)p.n1;
+                            const uint32_t d0 = tmem + (uint32_t)(st * kStageCols);
+                            if (phase == 0) {
+                                // D[row, key] for every row block: A = Q rows, B = the unit's keys
+                                for (int rb = 0; rb < p.nrb; ++rb) {
+                                    const uint64_t qd = ptx::sw128_kmajor_desc(q_addr + rb * 128 * 128);
+                                    const uint64_t kd = ptx::sw128_kmajor_desc(kbase + j * p.nk0 * 128);
 #pragma unroll
-                            for (int ks = 0; ks < D / 16; ++ks) {
-                                const uint32_t koff = (uint32_t)((ks >> 2) * kHalfTile + (ks & 3) * 32) >> 4;
-                                const uint32_t qoff = ((ks >> 2) * qhalf + (ks & 3) * 32) >> 4;
-                                const uint64_t kd = kdesc0 + koff;
-                                if (first_chunk)
-                                    ptx::mma_bf16_ss(d0, kd, qdesc0 + qoff, idesc1a, ks > 0);
-                                if (second_chunk)
-                                    ptx::mma_bf16_ss(d0 + n2_col, kd, qdesc0 + qoff + (uint32_t)(p.n1 * 128 >> 4),
-                                                     idesc1b, ks > 0);
-                                KVP_MSTAMP(kit, 3 + (ks & 7));
+                                    for (int ks = 0; ks < D / 16; ++ks) {
+                                        const uint32_t qo = ((ks >> 2) * qhalf + (ks & 3) * 32) >> 4;
+                                        const uint32_t ko = ((ks >> 2) * kHalfTile + (ks & 3) * 32) >> 4;
+                                        ptx::mma_bf16_ss(d0 + rb * p.nk0, qd + qo, kd + ko, idesc0, ks > 0);
+                                    }
+                                }
+                            } else {
+                                // D[key, row] for one part of the query rows: A = keys, B = Q rows
+                                const int np = j == p.p1 - 1 ? p.rows16 - j * p.n1 : p.n1;
+                                const uint32_t idesc1 = ptx::idesc_bf16_f32(128, np);
+                                const uint64_t qd = ptx::sw128_kmajor_desc(q_addr + j * p.n1 * 128);
+                                const uint64_t kd = ptx::sw128_kmajor_desc(kbase);
+#pragma unroll
+                                for (int ks = 0; ks < D / 16; ++ks) {
+                                    const uint32_t qo = ((ks >> 2) * qhalf + (ks & 3) * 32) >> 4;
+                                    const uint32_t ko = ((ks >> 2) * kHalfTile + (ks & 3) * 32) >> 4;
+                                    ptx::mma_bf16_ss(d0, kd + ko, qd + qo, idesc1, ks > 0);
+                                }
                             }
                             ptx::mma_commit(&sb->accfull[st]);
                         }
                         if (!ok) break;
                         ptx::mma_commit(&sb->kempty[s]);
-                        KVP_TSTAMP(kit, 3);
-                        KVP_MSTAMP(kit, 11);
-                        ++ait;
+                        KVP_TSTAMP(phase * n + i, 3);
                     }
                     if (!ok) break;
-                    // release the query tile when the next segment loads another head's
+                    // release the query rows when the next segment loads another head's
                     {
                         RunIter peek = it;
                         int nh = -1;
@@ -570,185 +513,145 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 }
                 KVP_STAMP(3 + phase);
             }
-            // all MMAs issued by this thread have completed before TMEM is released
+            // every MMA issued by this thread completes before TMEM is released, also when
+            // the CTA unwinds
             ptx::mma_commit(&sb->fin);
-            wait_phase(&sb->fin, 0, sb, p.err, kErrWaitMma);
+            drain_wait(&sb->fin, 0);
+        }
+    } else if (warp < kWarpEpi) {
+        // ------------------------------------------------------------ S2: max |V| per key
+        const int k2 = threadIdx.x - 32 * kWarpS2;          // 0 .. 63: keys k2 and k2 + 64
+        bool ok = true;
+        for (int i = 0; i < n && ok; ++i) {
+            const int jv = i % p.nv1, vuse = i / p.nv1;
+            if (!(ok = wait_phase(&sb->vfull[jv], vuse & 1, sb, p, kErrWaitS2))) break;
+            const uint8_t* vt = Slots + (p.nk1 + jv) * kSlotBytes;
+            const float ra = row_absmax<D>(vt + k2 * (D * 2), lane);
+            const float rb = row_absmax<D>(vt + (k2 + 64) * (D * 2), lane);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sb->vempty[jv]);
+            const int e = i & (kS2Bufs - 1), use = i / kS2Bufs;
+            if (!(ok = wait_phase(&sb->s2empty[e], (use & 1) ^ 1, sb, p, kErrWaitS2))) break;
+            s2buf[e * kTile + k2] = ra;
+            s2buf[e * kTile + k2 + 64] = rb;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sb->s2full[e]);
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - 64;                  // 0 .. kEpiThreads-1
-        const int wg = et >> 7;                           // epilogue group = TMEM stage
+        const int et = threadIdx.x - 32 * kWarpEpi;      // 0 .. kEpiThreads-1
+        const int eg = et >> 7;                           // epilogue group
         const int quarter = warp & 3;                     // TMEM lane quarter of this warp
-        const int lrow = quarter * 32 + lane;             // lane: query row (phase 0) / key (phase 1)
-        const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);   // this warp's lanes
+        const int lq = quarter * 32 + lane;               // lane: query row (phase 0) / key (phase 1)
+        const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
         const int window0 = p.L - p.w;                    // first window position
-        // columns (query rows) this group's TMEM stage holds: all rows when the groups
-        // alternate tiles, one half each when every tile is split across both stages
-        const int col0 = (p.split && wg == 1) ? p.n1 : 0;
-        const int ncols = p.split ? (wg == 0 ? p.n1 : p.rows - p.n1) : p.rows;
-        const int nch = (ncols + 31) >> 5;
-        const int warp8 = et >> 5;                        // epilogue warp 0..7
-        float* cwp = cw_all + warp8 * p.cw_stride;        // this warp's row offsets
-        int ait = 0;
         uint32_t epi_phase = 0;
         bool ok = true;
-        // ---- phase 0: per query row, each warp's running offset and sum of 2^(t - offset)
-        //      over its keys (thread = key, TMEM columns = query rows)
+        // ---- phase 0: per query row, the running offset and sum of 2^(t - m) over the keys
+        //      of this group's units (thread = row, TMEM columns = keys)
         {
+            // last visible key of this thread's row in each row block
+            int lim[4];
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb) lim[rb] = window0 + (rb * 128 + lq) % p.w;
+            // chunks of a unit that hold rows of this warp: all rows of a row block
+            // are live or none, and live chunks are a prefix of the unit's four
+            const int rbl = p.rows > quarter * 32 ? min(p.nrb, (p.rows - quarter * 32 + 127) / 128) : 0;
+            const int nl = min(4, rbl << p.lg_cpb);
+            const int cmask = (1 << p.lg_cpb) - 1;
             RunIter it(t0, t1, p.tiles_per_head);
             int head;
             long long a, b;
+            int unit = 0, i = 0;
             while (ok && it.next(head, a, b)) {
-                float lw[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                bool first_tile = true;
-                for (long long t = a; t < b && ok; ++t, ++ait) {
-                    if (!p.split && (ait & 1) != wg) continue;       // the other group's tile
-                    uint32_t parity;
-                    const int st = acc_stage(p.split, p.spg, ait, wg, parity);
-                    const uint32_t tstage = tlane + (uint32_t)(st * p.stage_cols);
-                    if (!(ok = wait_phase(&sb->accfull[st], parity, sb, p.err, kErrWaitEpi))) break;
-                    if (lrow == 0) KVP_TSTAMP(ait, 4);
-                    ptx::tc_fence_after();
-                    const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
-                    const int j = key0 + lrow;                       // this thread's key
-                    const int jw = j - window0;                      // > 0 only inside the window
-                    // masks, needed only by warps holding window keys and by a ragged last chunk
-                    // masks: window keys (query rows before the key) and columns past the
-                    // group's last; only warps holding window keys or a ragged last chunk
-                    // need them, which the warp decides as a whole
-                    const bool masked = __any_sync(0xffffffffu, jw > 0) || (ncols & 31);
-                    auto mask_chunk = [&](float (&v)[32], int c) {
-                        if (jw > 0) {
+                float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                float l[4] = {0.f, 0.f, 0.f, 0.f};
+                for (long long t = a; t < b && ok; ++t, ++i) {
+                    const int key_t = (int)(t - (long long)head * p.tiles_per_head) * kTile;
+                    for (int j = 0; j < p.u0; ++j, ++unit) {
+                        if ((unit & 1) != eg) continue;      // the other group's unit
+                        const int st = unit & (kStages - 1);
+                        if (!(ok = wait_phase(&sb->accfull[st], (unit / kStages) & 1, sb, p, kErrWaitEpi))) break;
+                        if (lq == 0) KVP_TSTAMP(i, 4);
+                        ptx::tc_fence_after();
+                        const int kbase = key_t + j * p.nk0;
+                        const uint32_t tst = tlane + (uint32_t)(st * kStageCols);
+                        // chunk c: TMEM columns [32c, 32c + 32) of the stage, row block c >> lg_cpb,
+                        // keys kbase + 32 (c & cmask) + e
+                        auto proc = [&](float (&v)[32], int c) {
+                            const int rb = c >> p.lg_cpb;
+                            const int j0 = kbase + ((c & cmask) << 5);
+                            if (j0 + 31 > window0) {         // window or ragged keys: mask per row
+                                const int rel = pick4(lim, rb) - j0;
 #pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                if (jw > (int)wpos[col0 + c * 32 + e]) v[e] = -INFINITY;
-                        }
-                        if ((c + 1) * 32 > ncols) {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                if (c * 32 + e >= ncols) v[e] = -INFINITY;
-                        }
-                    };
-                    // A head's first tile takes each row's offset from the warp's first key
-                    // (any offset within ~100 of a row's maximum keeps every exponential
-                    // finite; farther ones are caught by the overflow path).
-                    auto set_offsets = [&](const float (&v)[32], int c) {
-                        if (lane == 0) {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                cwp[c * 32 + e] = v[e] == -INFINITY ? -1e30f : v[e] * p.scale2;
-                        }
-                    };
-                    // Two chunks at a time so that their exponentials and shuffles interleave;
-                    // an odd last chunk is paired with an empty one.
-                    float x[32], y[32];
-                    __syncwarp();
-                    ptx::tmem_ld_32x32b_x32(tstage, x);
-                    ptx::tmem_ld_wait(x);
-#pragma unroll 1
-                    for (int c = 0; c < nch; c += 2) {
-                        const bool pair = c + 1 < nch;
-                        if (pair) {
-                            __syncwarp();
-                            ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
-                            ptx::tmem_ld_wait(y);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) y[e] = -INFINITY;
-                        }
-                        if (masked) {
-                            mask_chunk(x, c);
-                            if (pair) mask_chunk(y, c + 1);
-                        }
-                        if (first_tile) {
-                            __syncwarp();
-                            set_offsets(x, c);
-                            if (pair) set_offsets(y, c + 1);
-                            __syncwarp();
-                        }
-                        lse_pair_fast(x, y, cwp + c * 32, pair ? cwp + c * 32 + 32 : cwp + c * 32, p.scale2);
-                        float s0 = warp_reduce_scatter32<false>(x);
-                        float s1 = warp_reduce_scatter32<false>(y);
-                        float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-                        for (int cc = 0; cc < 8; cc += 2)
-                            if (cc == c) {
-                                l0 = lw[cc];
-                                l1 = lw[cc + 1];
+                                for (int e = 0; e < 32; ++e)
+                                    if (e > rel) v[e] = -INFINITY;
                             }
-                        if (__any_sync(0xffffffffu, !(s0 < INFINITY) || !(s1 < INFINITY))) {
-                            // rare: a logit far above its row's offset; raise, redo
-                            float2 r = lse_chunk_slow(tstage + c * 32, c * 32, ncols, col0, jw, false,
-                                                      cwp + c * 32, wpos, p.scale2, l0);
-                            s0 = r.x;
-                            l0 = r.y;
-                            if (pair) {
-                                r = lse_chunk_slow(tstage + (c + 1) * 32, (c + 1) * 32, ncols, col0, jw,
-                                                   false, cwp + (c + 1) * 32, wpos, p.scale2, l1);
-                                s1 = r.x;
-                                l1 = r.y;
-                            }
-                        }
-#pragma unroll
-                        for (int cc = 0; cc < 8; cc += 2)
-                            if (cc == c) {
-                                lw[cc] = l0 + s0;
-                                if (pair) lw[cc + 1] = l1 + s1;
-                            }
-                        if (c + 2 < nch) {
+                            float mr = pick4(m, rb), lr = pick4(l, rb);
+                            lse_chunk(v, p.scale2, mr, lr);
+                            put4(m, rb, mr);
+                            put4(l, rb, lr);
+                        };
+                        if (nl > 0) {
+                            float x[32], y[32];
                             __syncwarp();
-                            ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
+                            ptx::tmem_ld_32x32b_x32(tst, x);
                             ptx::tmem_ld_wait(x);
+#pragma unroll 1
+                            for (int c = 0; c < nl; c += 2) {
+                                const bool h1 = c + 1 < nl, h2 = c + 2 < nl;
+                                if (h1) {
+                                    __syncwarp();
+                                    ptx::tmem_ld_32x32b_x32(tst + (c + 1) * 32, y);
+                                }
+                                proc(x, c);
+                                if (h1) {
+                                    ptx::tmem_ld_wait(y);
+                                    if (h2) {
+                                        __syncwarp();
+                                        ptx::tmem_ld_32x32b_x32(tst + (c + 2) * 32, x);
+                                    }
+                                    proc(y, c + 1);
+                                    if (h2) ptx::tmem_ld_wait(x);
+                                }
+                            }
                         }
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&sb->accempty[st]);
+                        if (lq == 0) KVP_TSTAMP(i, 5);
                     }
-                    first_tile = false;
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[st]);
-                    if (lrow == 0) KVP_TSTAMP(ait, 5);
                 }
                 if (!ok) break;
-                // Combine the warps' (offset, sum) of every row inside the CTA, then publish
-                // one slot per row. The staging buffer aliases the offsets, so each lane
-                // first takes its own offsets into registers.
-                float cwr[8];
+                // Combine the two groups' (m, l) of every row, then publish one slot per row.
+                if (!(ok = epi_sync(sb, epi_phase, p))) break;   // stage0 free again
+                if (eg == 1) {
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const int n = cc * 32 + lane;
-                    cwr[cc] = (n < ncols) ? cwp[n] : 0.f;
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const int r = rb * 128 + lq;
+                        if (rb < p.nrb && r < p.rows) stage0[r] = make_float2(m[rb], l[rb]);
+                    }
                 }
-                if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
-                float2* stage = reinterpret_cast<float2*>(cw_all) + warp8 * p.cw_stride;
+                if (!(ok = epi_sync(sb, epi_phase, p))) break;
+                if (eg == 0) {
+                    const long long first = (long long)head * p.tiles_per_head;
+                    const int slot = (int)blockIdx.x - owner_of(first, T, p.grid, p.tiles_per_head, p.cph);
+                    const int r0 = group_row0(head);
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const int n = cc * 32 + lane;
-                    if (n < ncols)
-                        stage[n] = first_tile ? make_float2(-INFINITY, 0.f) : make_float2(cwr[cc], lw[cc]);
-                }
-                if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
-                const long long first = (long long)head * p.tiles_per_head;
-                const int slot = (int)blockIdx.x - owner_of(first, T, p.grid, p.tiles_per_head, p.cph);
-                const int r0 = group_row0(head);
-                for (int r = et; r < p.rows; r += kEpiThreads) {
-                    // warps holding row r: all eight, or the four of the group owning it
-                    const int g = (p.split && r >= p.n1) ? 1 : 0;
-                    const int n = r - (g ? p.n1 : 0);
-                    const int w_lo = p.split ? 4 * g : 0, w_hi = p.split ? 4 * g + 4 : 8;
-                    float M = -INFINITY, S = 0.f;
-                    for (int w = w_lo; w < w_hi; ++w) {
-                        const float2 ml = reinterpret_cast<const float2*>(cw_all)[w * p.cw_stride + n];
-                        if (ml.y == 0.f) continue;
-                        if (ml.x > M) {
-                            S = S * ptx::ex2(M - ml.x) + ml.y;
-                            M = ml.x;
-                        } else {
-                            S += ml.y * ptx::ex2(ml.x - M);
+                    for (int rb = 0; rb < 4; ++rb) {
+                        const int r = rb * 128 + lq;
+                        if (rb < p.nrb && r < p.rows) {
+                            const float2 o = stage0[r];
+                            const float M = fmaxf(m[rb], o.x);
+                            float S = 0.f;
+                            if (M != -INFINITY) S = l[rb] * ptx::ex2(m[rb] - M) + o.y * ptx::ex2(o.x - M);
+                            if (KVP_CHECK(slot >= 0 && slot < p.maxslots, 202, slot, head))
+                                p.part[(size_t)(r0 + r) * p.maxslots + slot] = make_float2(M, S);
                         }
                     }
-                    if (KVP_CHECK(slot >= 0 && slot < p.maxslots, 202, slot, head))
-                        p.part[(size_t)(r0 + r) * p.maxslots + slot] = make_float2(M, S);
+                    __threadfence();
                 }
-                if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
+                if (!(ok = epi_sync(sb, epi_phase, p))) break;
                 if (et == 0) {
                     __threadfence();
                     atomicAdd(p.done + head, 1u);
@@ -756,24 +659,24 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             }
         }
         if (et == 0) KVP_STAMP(5);
-        // ---- phase 1: scores
+        // ---- phase 1: scores (thread = key, TMEM columns = query rows)
         {
             bool first_seg = true;
             RunIter it(t0, t1, p.tiles_per_head);
             int head;
             long long a, b;
-            int pt = 0;                                   // phase 1 tile counter (V ring, handoff)
+            int unit = 0, i = 0;
             while (ok && it.next(head, a, b)) {
                 const long long first = (long long)head * p.tiles_per_head;
                 const int touch = owner_of(first + p.tiles_per_head - 1, T, p.grid, p.tiles_per_head, p.cph) -
-                                  owner_of(first, T, p.grid, p.tiles_per_head, p.cph) + 1;
+                                  owner_of(first, T, p.grid, p.tiles_per_head, p.cph) + 1 + p.extra_peers;
                 // the previous head's lse2 is no longer in use
-                if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
+                if (!(ok = epi_sync(sb, epi_phase, p))) break;
                 if (et == 0) {
                     const uint64_t ts = ptx::globaltimer_ns();
                     while (ptx::ld_acquire_u32(p.done + head) < (uint32_t)touch) {
                         if (*(volatile int*)&sb->abort_flag) break;
-                        if (ptx::globaltimer_ns() - ts > kWaitLimitNs) {
+                        if (ptx::globaltimer_ns() - ts > p.wait_limit_ns) {
                             atomicCAS(p.err, 0, kErrWaitPeers);
                             *(volatile int*)&sb->abort_flag = 1;
                             break;
@@ -781,7 +684,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         __nanosleep(128);
                     }
                 }
-                if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
+                if (!(ok = epi_sync(sb, epi_phase, p))) break;
                 if (et == 0 && first_seg) KVP_STAMP(6);
                 first_seg = false;
                 if (*(volatile int*)&sb->abort_flag) {
@@ -789,7 +692,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     break;
                 }
                 const int r0 = group_row0(head);
-                const int nslots = touch * kSlotsPerCta;
+                const int nslots = (touch - p.extra_peers) * kSlotsPerCta;
                 // Two threads per row, each over every other slot: first the row's
                 // maximum, then the sum of l 2^(m - max); every load and term independent.
                 for (int base = 0; base < 2 * p.rows; base += kEpiThreads) {
@@ -815,102 +718,86 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     S += __shfl_xor_sync(0xffffffffu, S, 1);
                     if (r < p.rows && (r2 & 1) == 0) lse2[r] = M + __log2f(S);
                 }
-                if (!(ok = epi_sync(sb, epi_phase, p.err))) break;
-                for (long long t = a; t < b && ok; ++t, ++ait, ++pt) {
-                    const bool mine = p.split || (ait & 1) == wg;
-                    if (!mine) continue;
-                    const bool reads_v = !p.split || wg == 0;
-                    const int key0 = (int)(t - first) * kTile;
-                    const int j = key0 + lrow;
-                    float s2v = 0.f;
-                    if (reads_v) {
-                        // S2: max |V[j, :]| from the staged tile, 16-byte pieces in a
-                        // rotated order per lane (conflict-free shared-memory reads)
-                        const int jv = pt % p.nv1;
-                        if (!(ok = wait_phase(&sb->vfull[jv], (pt / p.nv1) & 1, sb, p.err, kErrWaitEpi))) break;
-                        if (lrow == 0) KVP_TSTAMP(ait, 7);
-                        const uint4* vrow = (const uint4*)(Slots + (p.nk1 + jv) * kSlotBytes + lrow * (D * 2));
-                        constexpr int kPieces = D * 2 / 16;
-                        uint32_t mx = 0;
-#pragma unroll
-                        for (int c = 0; c < kPieces; ++c) {
-                            const uint4 x = vrow[(c + lane) & (kPieces - 1)];
-                            mx = bf16x2_absmax(mx, x.x & 0x7FFF7FFFu);
-                            mx = bf16x2_absmax(mx, x.y & 0x7FFF7FFFu);
-                            mx = bf16x2_absmax(mx, x.z & 0x7FFF7FFFu);
-                            mx = bf16x2_absmax(mx, x.w & 0x7FFF7FFFu);
-                        }
-                        s2v = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
+                if (!(ok = epi_sync(sb, epi_phase, p))) break;
+                for (long long t = a; t < b && ok; ++t, ++i) {
+                    const int j = (int)(t - first) * kTile + lq;     // this thread's key
+                    const int jw = j - window0;                      // > 0 only inside the window
+                    // masks (window keys) are decided per warp: TMEM loads are warp-collective,
+                    // so every lane takes the same path
+                    const bool win = __any_sync(0xffffffffu, jw > 0);
+                    float acc = 0.f;
+                    bool mine = false;
+                    for (int pp = 0; pp < p.p1; ++pp, ++unit) {
+                        if ((unit & 1) != eg) continue;
+                        mine = true;
+                        const int st = unit & (kStages - 1);
+                        const int use = ring_uses(st, kStages, U0) + unit / kStages;
+                        if (!(ok = wait_phase(&sb->accfull[st], use & 1, sb, p, kErrWaitEpi))) break;
+                        if (lq == 0) KVP_TSTAMP(n + i, 4);
+                        ptx::tc_fence_after();
+                        const uint32_t tst = tlane + (uint32_t)(st * kStageCols);
+                        const int col0 = pp * p.n1;
+                        const int ncols = min(p.n1, p.rows - col0);
+                        const int nch = (ncols + 31) >> 5;
+                        auto proc = [&](const float (&v)[32], int c) {
+                            const int nrem = ncols - c * 32;
+                            acc += s1_chunk(v, lse2 + col0 + c * 32, wpos + col0 + c * 32,
+                                            win || nrem < 32, jw, nrem, p.scale2);
+                        };
+                        float x[32], y[32];
                         __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&sb->vempty[jv]);
-                    }
-                    // S1 over this group's columns
-                    uint32_t parity;
-                    const int st = acc_stage(p.split, p.spg, ait, wg, parity);
-                    const uint32_t tstage = tlane + (uint32_t)(st * p.stage_cols);
-                    if (!(ok = wait_phase(&sb->accfull[st], parity, sb, p.err, kErrWaitEpi))) break;
-                    if (lrow == 0) KVP_TSTAMP(ait, 4);
-                    ptx::tc_fence_after();
-                    const int jw = j - window0;                     // > 0 only inside the window
-                    const int col0 = (p.split && wg == 1) ? p.n1 : 0;        // first query row
-                    const int ncols = p.split ? (wg == 0 ? p.n1 : p.rows - p.n1) : p.rows;
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                    // masks (window keys, a ragged last chunk) are decided per warp: TMEM loads
-                    // are warp-collective, so every lane takes the same loop
-                    const bool masked = __any_sync(0xffffffffu, jw > 0) || (ncols & 31);
-                    auto s1_chunk = [&](const float (&v)[32], int c) {
-                        if (masked)
-                            s1_chunk_masked(v, lse2 + col0 + c * 32, wpos + col0 + c * 32, jw, ncols - c * 32,
-                                            p.scale2, a0, a1, a2, a3);
-                        else
-                            s1_chunk_fast(v, lse2 + col0 + c * 32, p.scale2, a0, a1, a2, a3);
-                    };
-                    float x[32], y[32];
-                    __syncwarp();
-                    ptx::tmem_ld_32x32b_x32(tstage, x);
-                    ptx::tmem_ld_wait(x);
-                    for (int c = 0; c < nch; c += 2) {
-                        const bool has1 = c + 1 < nch, has2 = c + 2 < nch;
-                        if (has1) {
-                            __syncwarp();
-                            ptx::tmem_ld_32x32b_x32(tstage + (c + 1) * 32, y);
-                        }
-                        s1_chunk(x, c);
-                        if (has1) {
-                            ptx::tmem_ld_wait(y);
-                            if (has2) {
+                        ptx::tmem_ld_32x32b_x32(tst, x);
+                        ptx::tmem_ld_wait(x);
+#pragma unroll 1
+                        for (int c = 0; c < nch; c += 2) {
+                            const bool h1 = c + 1 < nch, h2 = c + 2 < nch;
+                            if (h1) {
                                 __syncwarp();
-                                ptx::tmem_ld_32x32b_x32(tstage + (c + 2) * 32, x);
+                                ptx::tmem_ld_32x32b_x32(tst + (c + 1) * 32, y);
                             }
-                            s1_chunk(y, c + 1);
-                            if (has2) ptx::tmem_ld_wait(x);
+                            proc(x, c);
+                            if (h1) {
+                                ptx::tmem_ld_wait(y);
+                                if (h2) {
+                                    __syncwarp();
+                                    ptx::tmem_ld_32x32b_x32(tst + (c + 2) * 32, x);
+                                }
+                                proc(y, c + 1);
+                                if (h2) ptx::tmem_ld_wait(x);
+                            }
                         }
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&sb->accempty[st]);
+                        if (lq == 0) KVP_TSTAMP(n + i, 5);
                     }
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[st]);
-                    if (lrow == 0) KVP_TSTAMP(ait, 5);
-                    float s1v = (a0 + a1) + (a2 + a3);
-                    if (p.split) {
-                        // hand the second group's partial to the first
-                        const int cb = pt & 1;
-                        const uint32_t cpar = (pt >> 1) & 1;
-                        if (wg == 1) {
-                            if (!(ok = wait_phase(&sb->combempty[cb], cpar ^ 1, sb, p.err, kErrWaitEpi))) break;
-                            comb[cb * kTile + lrow] = s1v;
+                    if (!ok || !mine) continue;
+                    if (p.p1 > 1) {
+                        // the tile's rows are split over both groups: the group of the last part
+                        // finishes the tile, the other hands over its partial S1
+                        const int fin = (i * p.p1 + p.p1 - 1) & 1;
+                        const int cb = i & (kCombBufs - 1), cuse = i / kCombBufs;
+                        if (eg != fin) {
+                            if (!(ok = wait_phase(&sb->combempty[cb], (cuse & 1) ^ 1, sb, p, kErrWaitEpi))) break;
+                            comb[cb * kTile + lq] = acc;
                             __syncwarp();
                             if (lane == 0) ptx::mbar_arrive(&sb->combfull[cb]);
                             continue;
                         }
-                        if (!(ok = wait_phase(&sb->combfull[cb], cpar, sb, p.err, kErrWaitEpi))) break;
-                        s1v += comb[cb * kTile + lrow];
+                        if (!(ok = wait_phase(&sb->combfull[cb], cuse & 1, sb, p, kErrWaitEpi))) break;
+                        acc += comb[cb * kTile + lq];
                         __syncwarp();
                         if (lane == 0) ptx::mbar_arrive(&sb->combempty[cb]);
                     }
-                    if (j < p.L && KVP_CHECK(head < p.total_tiles / p.tiles_per_head, 201, head, j)) {
+                    const int e = i & (kS2Bufs - 1), suse = i / kS2Bufs;
+                    if (!(ok = wait_phase(&sb->s2full[e], suse & 1, sb, p, kErrWaitEpi))) break;
+                    const float s2v = s2buf[e * kTile + lq];
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&sb->s2empty[e]);
+                    if (j < p.L) {
                         const size_t o = (size_t)head * p.L + j;
-                        p.score[o] = s1v * s2v;
-                        if (p.s1) p.s1[o] = s1v;
+                        p.score[o] = acc * s2v;
+                        if (p.s1) p.s1[o] = acc;
                         if (p.s2) p.s2[o] = s2v;
                     }
                 }
@@ -918,13 +805,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         }
     }
 
-    if (threadIdx.x == 64) KVP_STAMP(7);
-#ifdef KVP_TRACE
-    if (threadIdx.x == 64 && blockIdx.x < 4) {
-        g_kvp_ttrace[blockIdx.x][63][2] = clock64();
-        g_kvp_ttrace[blockIdx.x][63][3] = ptx::globaltimer_ns();
-    }
-#endif
+    if (threadIdx.x == 32 * kWarpEpi) KVP_STAMP(7);
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -973,6 +854,11 @@ struct Launch {
     size_t smem;
 };
 
+// Fault injection for the tests of a debug build: peers a head waits for that never
+// arrive, and the limit of every wait. Release builds keep the defaults.
+int g_extra_peers = 0;
+unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
 bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     Params& p = L->p;
     const int D = s.head_dim;
@@ -982,19 +868,16 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.rows = plan.rows;
     p.hq = s.hq;
     p.hkv = s.hkv;
-    p.D = D;
-    const int npad = (plan.rows + 15) / 16 * 16;
-    if (npad <= 256) {
-        p.n1 = npad;
-        p.n2 = 0;
-    } else {
-        p.n1 = (npad / 2 + 15) / 16 * 16;
-        p.n2 = npad - p.n1;
-    }
-    p.split = plan.rows > (int)kMaxStageCols ? 1 : 0;
-    // two 128-column stages per group when a tile's accumulator fits 128 columns
-    p.stage_cols = (!p.split && (plan.rows + 31) / 32 * 32 <= 128) ? 128 : 256;
-    p.spg = p.stage_cols == 128 ? 2 : 1;
+    // phase 0: row blocks of 128 query rows; a unit covers nk0 keys of every row block in
+    // 128 TMEM columns (4 chunks of 32 per thread)
+    p.nrb = (plan.rows + 127) / 128;
+    p.nk0 = p.nrb == 1 ? 128 : p.nrb == 2 ? 64 : 32;
+    p.u0 = kTile / p.nk0;
+    p.lg_cpb = p.nk0 == 128 ? 2 : p.nk0 == 64 ? 1 : 0;
+    // phase 1: the query rows in p1 parts of n1 (a multiple of 16, at most 128) rows
+    p.rows16 = (plan.rows + 15) / 16 * 16;
+    p.p1 = (p.rows16 + kStageCols - 1) / kStageCols;
+    p.n1 = ((p.rows16 + p.p1 - 1) / p.p1 + 15) / 16 * 16;
     p.tiles_per_head = plan.tiles_per_head;
     p.total_tiles = plan.total_tiles;
     // the planned cut, or a flat cut over the SMs of a smaller device
@@ -1013,55 +896,46 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     }
     p.maxslots = plan.maxslots;
     p.scale2 = 1.4426950408889634f / sqrtf((float)D);
-    const int qrows = (plan.rows + kQBoxRows - 1) / kQBoxRows * kQBoxRows;
-    p.qrows = qrows;
-    const uint32_t qbytes = (uint32_t)qrows * D * 2;
-    const uint32_t tile_bytes = (uint32_t)kTile * D * 2;
-    p.q_bytes = qbytes;
-    p.k_bytes = tile_bytes;
-    p.v_bytes = tile_bytes;
-    // shared memory: Q | K ring | V ring | lse2 + handoff | phase 0 row offsets | barriers
+    p.qrows = (plan.rows + kQBoxRows - 1) / kQBoxRows * kQBoxRows;
+    p.q_bytes = (uint32_t)p.qrows * D * 2;
+    p.tile_bytes = (uint32_t)kTile * D * 2;
+    p.extra_peers = g_extra_peers;
+    p.wait_limit_ns = g_wait_limit_ns;
+    // shared memory: Q | ring slots | lse2 | comb | s2buf | stage0 | wpos | barriers
     // (+1 KB to align the base)
-    const int group_cols = p.split ? std::max(p.n1, plan.rows - p.n1) : plan.rows;
-    p.cw_stride = (group_cols + 31) / 32 * 32;
-    const size_t cw_bytes = (size_t)(kEpiThreads / 32) * p.cw_stride * sizeof(float2);
-    // lse2[rows] (16-byte padded), then the split-mode handoff comb[2][128]
-    const size_t lse_floats = (size_t)((plan.rows + 3) / 4 * 4);
-    const size_t lse_bytes = (lse_floats + (p.split ? 2 * kTile : 0)) * sizeof(float);
+    const size_t lse_bytes = (size_t)((plan.rows + 3) / 4 * 4) * sizeof(float);
+    const size_t comb_bytes = (size_t)kCombBufs * kTile * sizeof(float);
+    const size_t s2_bytes = (size_t)kS2Bufs * kTile * sizeof(float);
+    const size_t stage_bytes = (size_t)plan.rows * sizeof(float2);
     const size_t wpos_bytes = (size_t)((plan.rows + 7) / 8 * 8) * sizeof(uint16_t);
-    const size_t fixed = std::max(lse_bytes, cw_bytes) + wpos_bytes + kBarBytes + 1024;
-    // As many ring slots as fit. Phase 1 splits them between K (read again, mostly from
-    // L2) and V (from HBM, so it gets the deeper share). Alternate-tile mode: both epilogue
-    // groups read V slots, each its own tiles; with an even number of V slots a group only
-    // ever waits on its own slots, one phase ahead at most (an odd count would make a group
-    // wait two phases ahead on a shared slot, where the parity test cannot tell the phases
-    // apart). Split mode: group 0 alone reads V.
-    if (qbytes + fixed > (size_t)kSmemLimit) return false;
-    // (a deeper ring measured slower on the 32K layer: 5 slots of 32 KiB gave a 1.5 us
-    // longer launch than 4)
-    p.ns = (int)std::min<size_t>(std::min<size_t>(kMaxSlots, kRingBytes / tile_bytes),
-                                 ((size_t)kSmemLimit - qbytes - fixed) / tile_bytes);
-    if (p.split) {
-        if (p.ns < 2) return false;
-        p.nv1 = p.ns / 2;
-    } else {
-        if (p.ns < 3) return false;
-        p.nv1 = p.ns >= 6 ? 4 : 2;
-    }
-    p.nk1 = p.ns - p.nv1;
-    const size_t total = qbytes + (size_t)p.ns * tile_bytes + fixed;
-    p.off_q = 0;
-    p.off_slots = qbytes;
-    // phase 0's row offsets / staging and phase 1's lse2 + handoff are never live at the
-    // same time (all epilogue threads pass a rendezvous between the phases): one region
-    p.off_cw = p.off_slots + p.ns * tile_bytes;
-    p.off_lse = p.off_cw;
-    p.off_wpos = p.off_cw + (uint32_t)std::max(lse_bytes, cw_bytes);
-    p.off_bar = p.off_wpos + (uint32_t)wpos_bytes;
+    const size_t fixed = lse_bytes + comb_bytes + s2_bytes + stage_bytes + wpos_bytes + kBarBytes + 1024;
+    if (p.q_bytes + fixed > (size_t)kSmemLimit) return false;
+    p.ns = (int)std::min<size_t>(kMaxSlots, ((size_t)kSmemLimit - p.q_bytes - fixed) / p.tile_bytes);
+    if (p.ns < 2) return false;
+    // phase 1: K comes again (mostly from L2), V from HBM gets the deeper share; a tile
+    // split into several parts holds its K slot longer, so one K slot can do
+    p.nk1 = (p.p1 > 1 && p.ns <= 3) ? 1 : 2;
+    p.nv1 = p.ns - p.nk1;
+    if (p.nv1 < 1) return false;
+    p.off_slots = p.q_bytes;
+    uint32_t off = p.off_slots + (uint32_t)p.ns * p.tile_bytes;
+    p.off_lse = off;
+    off += (uint32_t)lse_bytes;
+    p.off_comb = off;
+    off += (uint32_t)comb_bytes;
+    p.off_s2 = off;
+    off += (uint32_t)s2_bytes;
+    p.off_stage = off;
+    off += (uint32_t)stage_bytes;
+    p.off_wpos = off;
+    off += (uint32_t)wpos_bytes;
+    off = (off + 15) & ~15u;
+    p.off_bar = off;
+    off += (uint32_t)kBarBytes;
     static_assert(sizeof(SmemBars) <= kBarBytes, "barrier block");
     L->grid = p.grid;
-    L->smem = std::max(total, (size_t)kMinSmem);
-    return true;
+    L->smem = std::max<size_t>((size_t)off + 1024, (size_t)kMinSmem);
+    return L->smem <= (size_t)kSmemLimit;
 }
 
 }  // namespace
@@ -1104,7 +978,8 @@ cudaError_t launch_score(const kvp_shape& s, const Plan& plan, const uint16_t* q
         if (!make_map(&vmap, v, 3, dims, strides, vbox, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
-    if ((e = cudaMemsetAsync(ws + plan.off_done, 0, plan.off_part - plan.off_done, st)) != cudaSuccess)
+    // the error word, then the completion counters, start at zero on every call
+    if ((e = cudaMemsetAsync(ws + plan.off_err, 0, plan.off_part - plan.off_err, st)) != cudaSuccess)
         return e;
 
     void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const Params) =
@@ -1125,6 +1000,12 @@ cudaError_t launch_score(const kvp_shape& s, const Plan& plan, const uint16_t* q
 
 #ifdef KVP_CHECKS
 KVP_DEFINE_CHECK_READER(take_check_score)
+// Debug builds only: make every later scoring call wait for `extra_peers` completions per
+// head that never come, and give up any wait after `wait_limit_ns`.
+void set_fault(int extra_peers, unsigned long long wait_limit_ns) {
+    g_extra_peers = extra_peers;
+    g_wait_limit_ns = wait_limit_ns ? wait_limit_ns : kWaitLimitNs;
+}
 #endif
 #ifdef KVP_TRACE
 int take_trace(unsigned long long* out) {

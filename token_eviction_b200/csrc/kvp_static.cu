@@ -10,7 +10,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "kvp.h"
 #include "kvp_internal.cuh"
@@ -25,25 +24,14 @@ constexpr size_t kStaticScratchBytes = KVP_STATIC_SCRATCH_BYTES;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device, looked up once per device
-// (the array's name is only a host-side stand-in, not a device address).
+// Device address of the scratch array on the current device (the array's name is only a
+// host-side stand-in, not a device address). Looked up on every call: the lookup
+// allocates nothing, and a cached address could outlive the device's context.
 cudaError_t scratch_address(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_static_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = ptr;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = ptr;
     return cudaSuccess;
 }
 
@@ -66,9 +54,13 @@ extern "C" kvp_status kvp_score_static(const kvp_shape* shape, const uint16_t* q
     cudaError_t e = scratch_address(&scratch);
     if (e == cudaSuccess)
         e = launch_score(*shape, p, q_win, k, v, scratch, score, s1, s2, (cudaStream_t)stream);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return KVP_ERR_CUDA;
-    }
+    if (e != cudaSuccess) return record_cuda_error(e);
     return KVP_OK;
+}
+
+extern "C" kvp_status kvp_score_static_status(void* stream) {
+    void* scratch = nullptr;
+    const cudaError_t e = scratch_address(&scratch);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    return read_error_word(scratch, (cudaStream_t)stream);
 }
