@@ -50,6 +50,8 @@ def _get():
         lib.oracle_select.restype = i
         lib.oracle_compact.argtypes = [i, i, i, i, p, p, p, p, p]
         lib.oracle_compact.restype = i
+        lib.oracle_select_policy.argtypes = [i, i, i, i, i, i, i, i, p, p, p, p]
+        lib.oracle_select_policy.restype = i
         _lib = lib
     return _lib
 
@@ -91,6 +93,30 @@ def oracle_select(score, window: int, budget: int):
     if rc != 0:
         raise ValueError("oracle_select: bad window/budget")
     return idx
+
+
+MODE_PRODUCT, MODE_S1, MODE_S2 = 0, 1, 2
+
+
+def oracle_select_policy(s1, s2, window: int, budget: int, sinks: int = 0, kernel: int = 1,
+                         mode: int = MODE_PRODUCT, fp32_key: bool = False, want_key: bool = False):
+    """Kept positions [..., B] under a selection policy: sinks [0, s) always kept, S1
+    max-pooled with an odd kernel over the positions before the window, ranked by
+    pool(S1) * S2 (mode 0), pool(S1) (mode 1) or S2 (mode 2). ``fp32_key`` forms the key
+    in single precision with subnormals flushed, as the CUDA path does."""
+    s1 = np.ascontiguousarray(s1, dtype=np.float64)
+    s2 = np.ascontiguousarray(s2, dtype=np.float64)
+    assert s1.shape == s2.shape
+    lead, L = s1.shape[:-1], s1.shape[-1]
+    rows = int(np.prod(lead)) if lead else 1
+    idx = np.empty(lead + (budget,), dtype=np.int32)
+    key = np.full(s1.shape, np.nan) if want_key else None
+    rc = _get().oracle_select_policy(rows, L, window, budget, sinks, kernel, mode, int(fp32_key),
+                                     s1.ctypes.data, s2.ctypes.data, idx.ctypes.data,
+                                     None if key is None else key.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_select_policy: bad policy")
+    return (idx, key) if want_key else idx
 
 
 def oracle_compact(k, v, idx):

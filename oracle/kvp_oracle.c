@@ -29,9 +29,17 @@
  *
  * bf16 inputs arrive as their 16-bit patterns and are widened exactly to double.
  *
+ * Selection policies (oracle_select_policy), for the variants the pages name around the
+ * method: attention sinks (the CurDKV rebuttal page, "how our method processes the KV
+ * cache", step 5: the first s tokens are always kept), the ablations that rank by S1 alone
+ * or S2 alone (SlimKV page, the review of Section 4.6), and a pooling "kernel size" (same
+ * review; read here as SnapKV's 1-D max pooling of S1 over the positions before the window,
+ * the kernel centred on each position, positions past either end left out).
+ *
  * Parity pins (tests): sum_j S1 = G w; closed forms for identical keys and for a
  * single planted key; G = 1, w = 1 against a library softmax; brute force on tiny
- * inputs; selection against a library stable sort; gather against library indexing.
+ * inputs; selection against a library stable sort; gather against library indexing;
+ * pooling against a library sliding maximum and a planted spike.
  */
 #include <math.h>
 #include <stdint.h>
@@ -170,5 +178,69 @@ int oracle_compact(int rows, int L, int d, int B, const uint16_t* k, const uint1
             memcpy(k_out + ((size_t)r * B + t) * d, k + ((size_t)r * L + j) * d, sizeof(uint16_t) * d);
             memcpy(v_out + ((size_t)r * B + t) * d, v + ((size_t)r * L + j) * d, sizeof(uint16_t) * d);
         }
+    return 0;
+}
+
+/*
+ * Kept positions of every row under a selection policy.
+ *   s1, s2 [rows, L] double: S1 and S2 (Eq. 3 and Eq. 4)
+ *   sinks  s >= 0: positions [0, s) are always kept
+ *   kernel k >= 1, odd: S1 is max-pooled over [j - k/2, j + k/2] within [0, L - w)
+ *   mode   0: rank by pool(S1) * S2 (Eq. 5 with pooling); 1: by pool(S1); 2: by S2
+ *   fp32_key  nonzero: the ranking key is formed in single precision with subnormal
+ *             results flushed to zero (the arithmetic of the CUDA path), so that a
+ *             selection made on that path's own S1 and S2 can be compared exactly
+ *   idx    [rows, B] int32: [0, s), then the B - w - s highest keys among [s, L - w) (equal
+ *          keys: lower position first), then the window [L - w, L); ascending
+ *   key_out [rows, L] double (may be NULL): the ranking key of every position before the window
+ * Returns 0, or -1 on a bad policy (s + w > B, s > L - w, k even or < 1, mode outside 0..2).
+ */
+int oracle_select_policy(int rows, int L, int w, int B, int sinks, int kernel, int mode,
+                         int fp32_key, const double* s1, const double* s2, int32_t* idx,
+                         double* key_out) {
+    if (rows < 0 || w < 1 || w > L || B < w || B > L) return -1;
+    if (sinks < 0 || sinks + w > B || sinks > L - w) return -1;
+    if (kernel < 1 || kernel % 2 == 0 || mode < 0 || mode > 2) return -1;
+    const int n = L - w, half = kernel / 2;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < rows; ++r) {
+        const double* a = s1 + (size_t)r * L;
+        const double* v = s2 + (size_t)r * L;
+        double* key = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+        for (int j = 0; j < n; ++j) {
+            double pooled = a[j];
+            for (int t = j - half; t <= j + half; ++t)
+                if (t >= 0 && t < n && a[t] > pooled) pooled = a[t];
+            double k;
+            if (fp32_key) {
+                const float pf = (float)pooled, vf = (float)v[j];
+                float kf = mode == 0 ? pf * vf : mode == 1 ? pf : vf;
+                if (kf != 0.f && fabsf(kf) < 1.17549435e-38f) kf = 0.f;   /* flush subnormals */
+                k = (double)kf;
+            } else {
+                k = mode == 0 ? pooled * v[j] : mode == 1 ? pooled : v[j];
+            }
+            key[j] = k;
+            if (key_out) key_out[(size_t)r * L + j] = k;
+        }
+        const int nc = n - sinks, kk = B - w - sinks;
+        cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)(nc > 0 ? nc : 1));
+        unsigned char* keep = (unsigned char*)calloc((size_t)L, 1);
+        for (int j = 0; j < nc; ++j) {
+            c[j].s = key[sinks + j];
+            c[j].j = sinks + j;
+        }
+        qsort(c, (size_t)nc, sizeof(cand_t), by_score_then_pos);
+        for (int j = 0; j < sinks; ++j) keep[j] = 1;
+        for (int t = 0; t < kk; ++t) keep[c[t].j] = 1;
+        for (int j = n; j < L; ++j) keep[j] = 1;
+        int32_t* out = idx + (size_t)r * B;
+        int t = 0;
+        for (int j = 0; j < L; ++j)
+            if (keep[j]) out[t++] = j;
+        free(keep);
+        free(c);
+        free(key);
+    }
     return 0;
 }

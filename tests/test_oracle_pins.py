@@ -278,3 +278,86 @@ def test_permuting_keys_before_the_window_permutes_the_scores():
     np.testing.assert_array_equal(s2p[..., :n], s2[..., perm])
     np.testing.assert_allclose(sp[..., :n], s[..., perm], rtol=1e-10)
     np.testing.assert_allclose(s1p[..., n:], s1[..., n:], rtol=1e-10)
+
+
+# ---- selection policies: sinks, score modes, pooling kernel ---------------------------------
+
+def _library_policy_select(key, w, B, sinks):
+    """Kept set by numpy alone: [0, s), the B - w - s largest keys of [s, L - w) (stable on
+    position), the window."""
+    L = key.shape[-1]
+    n = L - w
+    cand = np.arange(sinks, n)
+    order = np.lexsort((cand, -key[sinks:n]))
+    chosen = cand[order[: B - w - sinks]]
+    return np.sort(np.concatenate([np.arange(sinks), chosen, np.arange(n, L)])).astype(np.int32)
+
+
+def test_policy_without_sinks_pooling_or_mode_is_the_plain_selection():
+    rng = np.random.default_rng(11)
+    s1, s2 = rng.random((3, 400)), rng.random((3, 400))
+    got = oracle.oracle_select_policy(s1, s2, 16, 90)
+    np.testing.assert_array_equal(got, oracle.oracle_select(s1 * s2, 16, 90))
+
+
+@pytest.mark.parametrize("sinks,kernel,mode", [(4, 1, 0), (0, 5, 0), (7, 7, 0), (3, 3, 1), (5, 1, 2),
+                                               (0, 1, 1), (16, 9, 0)])
+def test_policy_matches_library_pooling_and_sort(sinks, kernel, mode):
+    """Pooling against scipy's sliding maximum (positions past the ends left out), the
+    mode's key by numpy, the selection by numpy's stable lexsort."""
+    from scipy.ndimage import maximum_filter1d
+    rng = np.random.default_rng(100 + sinks + 10 * kernel + mode)
+    L, w, B = 333, 12, 80
+    s1, s2 = rng.random((2, L)), rng.random((2, L))
+    s1[:, 50:60] = 0.25                                  # a block of ties
+    got, key = oracle.oracle_select_policy(s1, s2, w, B, sinks, kernel, mode, want_key=True)
+    n = L - w
+    pooled = maximum_filter1d(s1[:, :n], size=kernel, axis=-1, mode="constant", cval=-np.inf)
+    want_key = pooled * s2[:, :n] if mode == 0 else pooled if mode == 1 else s2[:, :n]
+    np.testing.assert_array_equal(key[:, :n], want_key)
+    for r in range(2):
+        full = np.concatenate([want_key[r], np.zeros(w)])    # the window's keys are never ranked
+        np.testing.assert_array_equal(got[r], _library_policy_select(full, w, B, sinks))
+    assert (got[:, :sinks] == np.arange(sinks)).all()
+    assert (got[:, B - w:] == np.arange(n, L)).all()
+
+
+def test_pooling_spreads_a_planted_spike_over_the_kernel():
+    """S1 zero but one position: max pooling with kernel k turns it into a run of k equal
+    keys centred there (cut at the window), and a budget of exactly that run keeps it."""
+    L, w, k = 200, 10, 7
+    for j0, run in ((50, range(47, 54)), (2, range(0, 6)), (188, range(185, 190))):
+        s1 = np.zeros((1, L))
+        s1[0, j0] = 1.0
+        s2 = np.ones((1, L))
+        run = list(run)
+        got = oracle.oracle_select_policy(s1, s2, w, w + len(run), 0, k, 0)
+        np.testing.assert_array_equal(got[0], np.array(run + list(range(L - w, L)), dtype=np.int32))
+
+
+def test_sinks_are_kept_even_with_the_lowest_scores():
+    rng = np.random.default_rng(5)
+    s1 = rng.random((1, 300)) + 1.0
+    s1[0, :6] = 0.0                                      # the sinks score lowest of all
+    s2 = np.ones((1, 300))
+    got = oracle.oracle_select_policy(s1, s2, 8, 40, sinks=6)
+    assert got.shape == (1, 40)
+    assert (got[0, :6] == np.arange(6)).all() and (np.diff(got[0]) > 0).all()
+
+
+def test_single_precision_key_is_the_rounded_product():
+    rng = np.random.default_rng(9)
+    s1 = rng.random((2, 256)).astype(np.float32).astype(np.float64)
+    s2 = (rng.random((2, 256)) * 30).astype(np.float32).astype(np.float64)
+    s1[0, 3] = 1e-30                                     # product underflows to a subnormal
+    _, key = oracle.oracle_select_policy(s1, s2, 8, 64, fp32_key=True, want_key=True)
+    want = (s1.astype(np.float32) * s2.astype(np.float32)).astype(np.float64)
+    want[np.abs(want) < np.finfo(np.float32).tiny] = 0.0
+    np.testing.assert_array_equal(key[:, :248], want[:, :248])
+
+
+def test_bad_policies_raise():
+    s = np.ones((1, 50))
+    for kw in (dict(sinks=45), dict(sinks=-1), dict(kernel=4), dict(kernel=0), dict(mode=3)):
+        with pytest.raises(ValueError):
+            oracle.oracle_select_policy(s, s, 8, 40, **kw)
