@@ -102,6 +102,38 @@ KVP_API kvp_status kvp_score(const kvp_shape* shape, const uint16_t* q_win, cons
 KVP_API kvp_status kvp_select(const kvp_shape* shape, const float* score, int32_t* idx,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* Selection policies: the variants named around the method. */
+typedef enum {
+    KVP_RANK_PRODUCT = 0, /* pool(S1) * S2: Eq. 5 of SlimKV (with pooling when kernel > 1) */
+    KVP_RANK_S1 = 1,      /* pool(S1) alone: the SlimKV ablation without S2 (review of Sec. 4.6) */
+    KVP_RANK_S2 = 2       /* S2 alone: the SlimKV ablation without S1 (same review) */
+} kvp_rank_mode;
+
+typedef struct {
+    int32_t sinks;        /* s >= 0: positions [0, s) are always kept (attention sinks; CurDKV
+                             rebuttal, "how our method processes the KV cache", step 5) */
+    int32_t pool_kernel;  /* k, odd, 1 <= k <= 255: S1 is max-pooled over [j - k/2, j + k/2]
+                             within [0, L - w) before ranking (the "kernel size" of the SlimKV
+                             review of Sec. 4.6, read as SnapKV-style 1-D max pooling); 1: none */
+    int32_t mode;         /* a kvp_rank_mode */
+} kvp_policy;
+
+/*
+ * Kept positions under a policy: the first s positions, the B - w - s candidates of
+ * [s, L - w) with the highest keys (equal keys: lower position first), and the window
+ * [L - w, L), listed in ascending position order. The key of candidate j is formed in
+ * fp32 from S1 and S2 (as kvp_score writes them):
+ *   p_j = max of s1 over [j - k/2, j + k/2] within [0, L - w)
+ *   mode PRODUCT: p_j * s2_j (rounded to nearest, subnormal operands kept); S1: p_j; S2: s2_j
+ *   a key below the smallest normal fp32 counts as zero.
+ *   s1, s2  [b, hkv, L] fp32, non-negative; s1 may be NULL in mode S2, s2 in mode S1
+ *   idx     [b, hkv, B] int32 output
+ * Needs s + w <= B and s <= L - w (else KVP_ERR_SHAPE, as for a bad kernel or mode).
+ * No workspace: the call keeps its keys in shared memory.
+ */
+KVP_API kvp_status kvp_select_policy(const kvp_shape* shape, const kvp_policy* policy,
+                                     const float* s1, const float* s2, int32_t* idx, void* stream);
+
 /*
  * Compaction: k_out[b, h, t, :] = k[b, h, idx[b, h, t], :], the same for v; a bit copy.
  *   k, v          [b, hkv, L, d] bf16

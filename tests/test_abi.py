@@ -19,7 +19,8 @@ def declared_symbols():
 
 
 def test_header_declares_the_boundary():
-    assert {"kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact", "kvp_workspace_status",
+    assert {"kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_select_policy", "kvp_compact",
+            "kvp_workspace_status",
             "kvp_score_static", "kvp_score_static_status", "kvp_status_string",
             "kvp_last_cuda_error"} <= declared_symbols()
 
@@ -86,6 +87,31 @@ def test_host_side_argument_errors():
     assert m._lib.kvp_compact(ctypes.byref(sh), 16, 16, 16, 16, 8, None) == 3
     bad = m.make_shape(1, 32, 8, 128, 4096, 32, 8)
     assert m._lib.kvp_compact(ctypes.byref(bad), 16, 16, 16, 16, 16, None) == 2
+
+
+def test_policy_select_rejects_bad_policies_on_the_host():
+    import token_eviction_b200 as m
+    sh = m.make_shape(1, 32, 8, 128, 4096, 32, 256)
+
+    def call(sinks=0, kernel=1, mode=0, s1=16, s2=16, idx=16, shape=sh):
+        pol = m.make_policy(sinks, kernel, mode)
+        return m._lib.kvp_select_policy(ctypes.byref(shape), ctypes.byref(pol), s1, s2, idx, None)
+
+    assert call(kernel=2) == 2                # even kernel
+    assert call(kernel=0) == 2
+    assert call(kernel=257) == 2
+    assert call(mode=3) == 2
+    assert call(mode=-1) == 2
+    assert call(sinks=-1) == 2
+    assert call(sinks=225) == 2               # sinks + w > B
+    small = m.make_shape(1, 32, 8, 128, 64, 32, 64)
+    assert call(sinks=33, shape=small) == 2   # sinks > L - w
+    assert call(idx=None) == 1
+    assert call(s1=None) == 1                 # product needs S1
+    assert call(mode=1, s1=None) == 1
+    assert call(mode=2, s2=None) == 1
+    assert call(s1=24) == 3                   # misaligned
+    assert m._lib.kvp_select_policy(ctypes.byref(sh), None, 16, 16, 16, None) == 1
 
 
 def test_binding_validates_tensors_before_calling():

@@ -10,6 +10,7 @@ The functions carry the C names:
 * ``kvp_workspace_bytes(shape)``
 * ``kvp_score(shape, q_win, k, v, score, s1=None, s2=None, workspace=None, stream=None)``
 * ``kvp_select(shape, score, idx, workspace=None, stream=None)``
+* ``kvp_select_policy(shape, policy, s1, s2, idx, stream=None)``
 * ``kvp_compact(shape, k, v, idx, k_out, v_out, stream=None)``
 * ``kvp_workspace_status(workspace, stream=None)``
 * ``kvp_status_string(status)``
@@ -47,6 +48,18 @@ class KvpShape(ctypes.Structure):
                 % (self.batch, self.hq, self.hkv, self.head_dim, self.seq_len, self.window, self.budget))
 
 
+RANK_PRODUCT, RANK_S1, RANK_S2 = 0, 1, 2
+
+
+class KvpPolicy(ctypes.Structure):
+    """Mirror of ``kvp_policy``: sinks always kept, S1 max-pooling kernel, ranking mode."""
+    _fields_ = [("sinks", ctypes.c_int32), ("pool_kernel", ctypes.c_int32), ("mode", ctypes.c_int32)]
+
+
+def make_policy(sinks=0, pool_kernel=1, mode=RANK_PRODUCT) -> KvpPolicy:
+    return KvpPolicy(int(sinks), int(pool_kernel), int(mode))
+
+
 class KvpError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -69,6 +82,8 @@ def _load():
     lib.kvp_score.restype = ctypes.c_int
     lib.kvp_select.argtypes = [S, P, P, P, ctypes.c_size_t, P]
     lib.kvp_select.restype = ctypes.c_int
+    lib.kvp_select_policy.argtypes = [S, ctypes.POINTER(KvpPolicy), P, P, P, P]
+    lib.kvp_select_policy.restype = ctypes.c_int
     lib.kvp_compact.argtypes = [S, P, P, P, P, P, P]
     lib.kvp_compact.restype = ctypes.c_int
     lib.kvp_status_string.argtypes = [ctypes.c_int]
@@ -91,7 +106,8 @@ _lib = _load()
 # enqueues one small memset of its workspace counters.
 KERNELS_PER_LAYER = 3
 
-EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_compact", "kvp_workspace_status",
+EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_select_policy", "kvp_compact",
+            "kvp_workspace_status",
             "kvp_score_static", "kvp_score_static_status", "kvp_status_string", "kvp_last_cuda_error")
 
 
@@ -187,6 +203,20 @@ def kvp_select(shape, score, idx, workspace=None, stream=None):
                          _stream(stream))
     if st != KVP_OK:
         raise KvpError(st, "kvp_select")
+
+
+def kvp_select_policy(shape, policy, s1, s2, idx, stream=None):
+    """Kept positions under `policy` (a KvpPolicy, or a dict of make_policy's arguments):
+    sinks, then the best candidates by the policy's key, then the window; ascending."""
+    sh = _as_shape(shape)
+    pol = policy if isinstance(policy, KvpPolicy) else make_policy(**policy)
+    b, hkv, L, B = sh.batch, sh.hkv, sh.seq_len, sh.budget
+    p1 = _ptr(s1, "s1", torch.float32, (b, hkv, L), optional=pol.mode == RANK_S2)
+    p2 = _ptr(s2, "s2", torch.float32, (b, hkv, L), optional=pol.mode == RANK_S1)
+    pi = _ptr(idx, "idx", torch.int32, (b, hkv, B))
+    st = _lib.kvp_select_policy(ctypes.byref(sh), ctypes.byref(pol), p1, p2, pi, _stream(stream))
+    if st != KVP_OK:
+        raise KvpError(st, "kvp_select_policy")
 
 
 def kvp_compact(shape, k, v, idx, k_out, v_out, stream=None):

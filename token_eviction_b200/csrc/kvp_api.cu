@@ -47,60 +47,6 @@ cudaError_t allow_dynamic_smem(const void* func, size_t bytes) {
     return cudaSuccess;
 }
 
-static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-static bool shape_ok(const kvp_shape& s) {
-    if (s.batch < 1 || s.hkv < 1 || s.hq < 1 || s.hq % s.hkv != 0) return false;
-    if (s.head_dim != 64 && s.head_dim != 128) return false;
-    if (s.seq_len < 1 || s.window < 1 || s.window > s.seq_len) return false;
-    if (s.budget < s.window || s.budget > s.seq_len) return false;
-    if ((int64_t)(s.hq / s.hkv) * s.window > kMaxGroupRows) return false;
-    // element offsets of k/v stay well inside int64; row counts inside int32
-    if ((int64_t)s.batch * s.hkv > 65535) return false;  // grid y extent
-    if ((int64_t)s.batch * s.hkv * s.seq_len > INT32_MAX) return false;
-    if ((int64_t)s.batch * s.hq * s.window > INT32_MAX) return false;
-    if ((int64_t)s.batch * s.hkv * s.budget * 16 > INT32_MAX / 2) return false;  // gather pieces
-    return true;
-}
-
-bool plan_of(const kvp_shape& s, Plan* p) {
-    if (!shape_ok(s)) return false;
-    p->G = s.hq / s.hkv;
-    p->rows = p->G * s.window;
-    const long long units = (long long)s.batch * s.hkv;
-    p->tiles_per_head = (s.seq_len + 127) / 128;
-    const long long T = units * p->tiles_per_head;
-    if (T > INT32_MAX) return false;
-    p->total_tiles = (int)T;
-    const long long tph = p->tiles_per_head;
-    const long long flat_grid = std::min<long long>(kPlanGrid, T);
-    const long long cph = units <= kPlanGrid ? std::min<long long>(kPlanGrid / units, tph) : 0;
-    // head-aligned runs unless their longest run exceeds the flat cut's by more than
-    // what a change of head costs a flat run
-    const bool aligned = cph > 0 && (tph + cph - 1) / cph <= (T + flat_grid - 1) / flat_grid + kHeadSwitchTiles;
-    p->cph = aligned ? (int)cph : 0;
-    p->grid = aligned ? (int)(cph * units) : (int)flat_grid;
-    int slots = 0;
-    for (long long h = 0; h < units; ++h) {
-        const long long f = h * tph;
-        slots = std::max(slots, owner_of(f + tph - 1, T, p->grid, tph, p->cph) -
-                                    owner_of(f, T, p->grid, tph, p->cph) + 1);
-    }
-    p->maxslots = slots * kSlotsPerCta;
-    // the error word sits at offset 0 of every workspace, so that a status read needs no shape
-    size_t off = 0;
-    p->off_err = off;
-    off += 256;
-    p->off_done = off;
-    off += align_up((size_t)units * sizeof(uint32_t), 256);
-    p->off_part = off;
-    off += align_up((size_t)s.batch * s.hq * s.window * p->maxslots * sizeof(float2), 256);
-    p->off_select = off;
-    off += 256;
-    p->bytes = off;
-    return true;
-}
-
 }  // namespace kvp
 
 using namespace kvp;
@@ -163,6 +109,25 @@ extern "C" kvp_status kvp_select(const kvp_shape* shape, const float* score, int
     if (!aligned16(workspace)) return KVP_ERR_ALIGN;
     const cudaError_t e =
         launch_select(*shape, p, score, idx, (char*)workspace + p.off_select, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_failed(e);
+    return KVP_OK;
+}
+
+extern "C" kvp_status kvp_select_policy(const kvp_shape* shape, const kvp_policy* policy,
+                                        const float* s1, const float* s2, int32_t* idx, void* stream) {
+    if (!shape || !policy || !idx) return KVP_ERR_NULL;
+    const int mode = policy->mode;
+    if (mode < KVP_RANK_PRODUCT || mode > KVP_RANK_S2) return KVP_ERR_SHAPE;
+    if ((mode != KVP_RANK_S2 && !s1) || (mode != KVP_RANK_S1 && !s2)) return KVP_ERR_NULL;
+    Plan p;
+    if (!plan_of(*shape, &p)) return KVP_ERR_SHAPE;
+    const int k = policy->pool_kernel, sinks = policy->sinks;
+    if (k < 1 || k > 255 || k % 2 == 0) return KVP_ERR_SHAPE;
+    if (sinks < 0 || sinks + shape->window > shape->budget || sinks > shape->seq_len - shape->window)
+        return KVP_ERR_SHAPE;
+    if (!aligned16(s1) || !aligned16(s2) || !aligned16(idx)) return KVP_ERR_ALIGN;
+    const cudaError_t e = launch_select_policy(*shape, *policy, mode == KVP_RANK_S2 ? nullptr : s1,
+                                               mode == KVP_RANK_S1 ? nullptr : s2, idx, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_failed(e);
     return KVP_OK;
 }

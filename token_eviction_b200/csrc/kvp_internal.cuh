@@ -13,18 +13,22 @@ namespace kvp {
 constexpr int kMaxGroupRows = 512;
 
 // How a shape is cut into work: 128-key tiles of the flattened (sequence, KV head, key)
-// space dealt out in contiguous runs to the scoring kernel's CTAs, and the workspace
-// layout. A pure function of the shape, so kvp_workspace_bytes, kvp_score and
-// kvp_select agree. Runs are either aligned to the KV heads (every head cut into cph
-// runs of its own, so no CTA pays for a change of head) or, when that would leave too
-// many SMs idle, the flattened tiles cut evenly across all CTAs (cph = 0).
+// space dealt out to the scoring kernel's CTAs, and the workspace layout. A pure function
+// of the shape, so kvp_workspace_bytes, kvp_score and kvp_select agree.
+//   Head-aligned (cph > 0): every KV head is cut into cph parts of consecutive tiles, and
+//     each CTA takes nseg parts (segments) of different heads. With two segments a CTA
+//     sweeps phase 0 over both heads before phase 1 over either, so the wait for the
+//     first head's other CTAs overlaps the second head's phase 0.
+//   Flat (cph = 0, nseg = 1): the flattened tiles cut evenly across the CTAs, for shapes
+//     with more KV heads than SMs; a run may then cross heads.
 struct Plan {
     int G;               // query heads per KV head
     int rows;            // G * w: window queries per KV head
     int tiles_per_head;  // 128-key tiles per (sequence, KV head)
     int total_tiles;     // over all (sequence, KV head)
-    int grid;            // CTAs of the scoring kernel (one per SM, at most one per tile)
-    int cph;             // runs per KV head when runs are head-aligned; 0: flat runs
+    int grid;            // CTAs of the scoring kernel (one per SM)
+    int cph;             // parts per KV head when head-aligned; 0: flat runs
+    int nseg;            // segments per CTA (1 or 2 when head-aligned; 1 when flat)
     int maxslots;        // partial-softmax slots per query row (CTAs touching one head)
     size_t off_err;      // int: first device-side error code (0 = none); always offset 0
     size_t off_done;     // uint32 per (sequence, KV head): CTAs done with phase 0
@@ -42,27 +46,74 @@ constexpr int kSlotsPerCta = 1;
 
 bool plan_of(const kvp_shape& s, Plan* p);
 
-// Runs of the scoring kernel's CTAs over the T tiles (tph per KV head). Flat (cph = 0):
-// CTA c takes [floor(c T / grid), floor((c + 1) T / grid)). Head-aligned (cph > 0,
-// grid = cph * heads): CTA c takes part c % cph of head c / cph, the same cut within the
-// head's tph tiles.
-__host__ __device__ __forceinline__ long long run_begin(long long c, long long T, long long grid,
-                                                        long long tph, long long cph) {
-    if (cph > 0) return (c / cph) * tph + (c % cph) * tph / cph;
+// Flat runs over the T tiles: CTA c takes [floor(c T / grid), floor((c + 1) T / grid)).
+__host__ __device__ __forceinline__ long long run_begin(long long c, long long T, long long grid) {
     return c * T / grid;
 }
-// The CTA whose run holds tile t.
-__host__ __device__ __forceinline__ int owner_of(long long t, long long T, long long grid,
-                                                 long long tph, long long cph) {
-    if (cph > 0) return (int)((t / tph) * cph + ((t % tph + 1) * cph + tph - 1) / tph - 1);
+// The CTA whose flat run holds tile t.
+__host__ __device__ __forceinline__ int owner_of(long long t, long long T, long long grid) {
     return (int)(((t + 1) * grid + T - 1) / T - 1);
 }
 
+// Segment s of CTA c: tiles [b, e). Head-aligned: global part g = s * grid + c, of head
+// g / cph, part g % cph, the same cut within every head's tph tiles (grid * nseg =
+// cph * heads, so the two segments of a CTA lie in heads grid / cph apart). Flat: the run.
+__host__ __device__ __forceinline__ void segment_of(long long c, int s, long long T, long long grid,
+                                                    long long tph, long long cph, long long& b,
+                                                    long long& e) {
+    if (cph > 0) {
+        const long long g = s * grid + c, h = g / cph, part = g % cph;
+        b = h * tph + part * tph / cph;
+        e = h * tph + (part + 1) * tph / cph;
+    } else {
+        b = run_begin(c, T, grid);
+        e = run_begin(c + 1, T, grid);
+    }
+}
+// Slot of CTA c's partial among the CTAs touching head h (reached through segment s).
+__host__ __device__ __forceinline__ int slot_in_head(long long c, int s, long long h, long long T,
+                                                     long long grid, long long tph, long long cph) {
+    if (cph > 0) return (int)((s * grid + c) % cph);
+    return (int)(c - owner_of(h * tph, T, grid));
+}
+// Number of CTAs that touch head h.
+__host__ __device__ __forceinline__ int ctas_touching(long long h, long long T, long long grid,
+                                                      long long tph, long long cph) {
+    if (cph > 0) return (int)cph;
+    return owner_of(h * tph + tph - 1, T, grid) - owner_of(h * tph, T, grid) + 1;
+}
+
+// The same three in unsigned 32-bit arithmetic, for device code: the plan keeps
+// T * (kPlanGrid + 1) below 2^32 and cph <= kPlanGrid, so no product below overflows.
+__device__ __forceinline__ void segment_of_u32(uint32_t c, uint32_t s, uint32_t T, uint32_t grid,
+                                               uint32_t tph, uint32_t cph, uint32_t& b, uint32_t& e) {
+    if (cph > 0) {
+        const uint32_t g = s * grid + c, h = g / cph, part = g - h * cph;
+        b = h * tph + part * tph / cph;
+        e = h * tph + (part + 1) * tph / cph;
+    } else {
+        b = c * T / grid;
+        e = (c + 1) * T / grid;
+    }
+}
+__device__ __forceinline__ uint32_t owner_of_u32(uint32_t t, uint32_t T, uint32_t grid) {
+    return ((t + 1) * grid + T - 1) / T - 1;
+}
+__device__ __forceinline__ uint32_t slot_in_head_u32(uint32_t c, uint32_t s, uint32_t h, uint32_t T,
+                                                     uint32_t grid, uint32_t tph, uint32_t cph) {
+    if (cph > 0) return (s * grid + c) % cph;
+    return c - owner_of_u32(h * tph, T, grid);
+}
+__device__ __forceinline__ uint32_t ctas_touching_u32(uint32_t h, uint32_t T, uint32_t grid, uint32_t tph,
+                                                      uint32_t cph) {
+    if (cph > 0) return cph;
+    return owner_of_u32(h * tph + tph - 1, T, grid) - owner_of_u32(h * tph, T, grid) + 1;
+}
+
 // Tiles by which a head-aligned cut's longest run may exceed the flat cut's and still be
-// chosen. A run that changes head in mid-stream waits, at the start of its second head's
-// scoring pass, for that head's other runs and a fresh query block: on the 32K layer
-// (8 heads, 148 SMs) such runs ended about 16 us after the rest, while 15-tile aligned
-// runs ended within 3 us of each other.
+// chosen. A flat run that changes head in mid-stream waits, at the start of its second
+// head's scoring pass, for that head's other runs and a fresh query block: on the 32K layer
+// (8 heads, 148 SMs) such runs ended about 16 us after the rest.
 constexpr int kHeadSwitchTiles = 3;
 
 // Launchers (each returns the launch's cudaError_t).
@@ -71,6 +122,8 @@ cudaError_t launch_score(const kvp_shape& s, const Plan& p, const uint16_t* q, c
                          cudaStream_t st);
 cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score, int32_t* idx,
                           void* scratch, cudaStream_t st);
+cudaError_t launch_select_policy(const kvp_shape& s, const kvp_policy& pol, const float* s1,
+                                 const float* s2, int32_t* idx, cudaStream_t st);
 cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t* v,
                            const int32_t* idx, uint16_t* k_out, uint16_t* v_out, cudaStream_t st);
 

@@ -8,28 +8,36 @@
 // Window query i sits at position L - w + i and sees keys j <= L - w + i.
 //
 // A softmax row's denominator must be known before any key's S1 can be summed, so K is
-// swept twice; both sweeps run inside one kernel. Each CTA owns a contiguous run of
-// 128-key tiles of the flattened (sequence, KV head, tile) space.
+// swept twice; both sweeps run inside one kernel. Each CTA owns one or two segments of
+// consecutive 128-key tiles (of different KV heads, when two), and sweeps phase 0 over all
+// of them before phase 1, so that the wait for one head's other CTAs overlaps the next
+// head's phase 0.
 //   phase 0 (log-sum-exp; one query row per thread): tcgen05 computes
 //     D[row, key] = Q_group[row] . K_tile[key]  (M = 128 rows of one row block, N = keys),
 //     so each epilogue thread owns one query row (a TMEM lane) and keeps its running
 //     offset m and sum l = sum_j 2^(t_j - m) in registers, t = logit * log2(e) / sqrt(d).
-//     At the end of each KV head in its run a CTA publishes one (m, l) slot per row to
-//     the workspace and bumps the head's completion counter.
+//     At the end of each segment a CTA publishes one (m, l) slot per row to the workspace
+//     and bumps the head's completion counter.
 //   phase 1 (scores; one key per thread): the same tiles again (K now mostly from L2),
 //     with D[key, row] = K_tile[key] . Q_group[row]  (M = 128 keys, N = query rows).
 //     Before its first tile of a head a CTA waits (bounded) until every CTA touching the
 //     head has published, then merges the slots into lse2 = M + log2(sum_s l_s 2^(m_s-M))
 //     per row. Per tile each thread sums 2^(t - lse2) over its key's query rows: S1.
-//   S2 is reduced from each V tile, staged once in shared memory, by two warps of its own,
-//   so that V's arrival from HBM never stalls the exponentials.
-// Warp roles: warp 0 issues TMA loads (a ring of tile slots and the group's query rows),
-// warp 1 allocates TMEM and issues the MMAs from one thread, warps 2-3 reduce V tiles to
-// S2, and two epilogue warpgroups (warps 4-7 and 8-11, one TMEM lane quarter per warp)
-// read the accumulators. TMEM holds four accumulator stages of 128 columns; a tile's work
-// is cut into units of at most 128 columns (phase 0: a run of keys over every row block;
-// phase 1: a part of the query rows), unit k takes stage k % 4, and stage s belongs to
-// epilogue group s % 2.
+//   S2 comes from phase 1's V tiles (V streams from HBM beside phase 1's K, which comes
+//     mostly from L2: phase 0 streams K alone, so that K stays in L2). Each V tile is cut
+//     into 4 pieces of 32 keys; any warp that would otherwise wait claims the next piece
+//     (in order, through a shared counter) and reduces it into a ring of per-tile S2 rows
+//     in shared memory, which the tile's finishing warps read. No busy warp holds up the V
+//     stream, and the exponentials never wait for V.
+// Warp roles: warp 0 issues the TMA loads (a ring of tile slots in shared memory, and the
+// group's query rows); warp 1 allocates TMEM and issues the MMAs from one thread; warp 2
+// combines the epilogue groups' phase 0 sums and publishes them (so that no epilogue thread
+// waits on a global fence); warp 3 only reduces V pieces; four epilogue warpgroups (warps
+// 4-19, one TMEM lane quarter per warp) read the accumulators. TMEM holds four accumulator
+// stages of 128 columns, stage s belonging to epilogue group s. A tile's work is cut into
+// units of at most 128 columns (phase 0: a run of keys over every row block; phase 1: a
+// part of the query rows), and unit k takes stage k % 4, so four units are in flight and
+// each group has four units' time for one.
 // Every wait is bounded by a timer; a wait that gives up records an error code in the
 // workspace and the CTA unwinds without touching TMEM or shared memory still in use.
 #include <cuda.h>
@@ -49,17 +57,21 @@ namespace kvp {
 namespace {
 
 constexpr int kTile = 128;                        // keys per tile
-constexpr int kGroups = 2;                        // epilogue warpgroups
 constexpr int kStages = 4;                        // TMEM accumulator stages
+constexpr int kGroups = kStages;                  // epilogue warpgroups, one per stage
 constexpr int kStageCols = 128;                   // TMEM columns per stage
 constexpr uint32_t kTmemCols = kStages * kStageCols;
-constexpr int kWarpS2 = 2, kS2Warps = 2;          // warps that reduce V tiles to S2
-constexpr int kWarpEpi = kWarpS2 + kS2Warps;      // first epilogue warp
+constexpr int kWarpPub = 2;                       // the warp that publishes phase 0 sums
+constexpr int kWarpV = 3;                         // a warp that only reduces V pieces (and warp 2,
+                                                  // once it has published phase 0)
+constexpr int kWarpEpi = 4;                       // first epilogue warp
 constexpr int kEpiThreads = 128 * kGroups;
 constexpr int kThreads = 32 * kWarpEpi + kEpiThreads;
 constexpr int kMaxSlots = 8;                      // tile slots of the load ring
-constexpr int kS2Bufs = 4;                        // S2 hand-off buffers (one tile each)
-constexpr int kCombBufs = 2;                      // partial-S1 hand-off buffers
+constexpr int kCombBufs = 4;                      // partial-S1 hand-off buffers (one tile each)
+constexpr int kS2Ring = 8;                        // per-tile S2 rows in shared memory
+constexpr int kVPieces = 4;                       // pieces of 32 keys per V tile
+constexpr int kMaxParts = 4;                      // phase 1 parts per tile (512 rows / 128)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s on any single wait
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMinSmem = 116 * 1024;              // forces one CTA per SM (TMEM is taken whole)
@@ -69,11 +81,14 @@ constexpr float kSumLimit = 1.8446744e19f;        // 2^64: a chunk sum above it 
 
 #ifdef KVP_TRACE
 // Debug builds only: %globaltimer stamps per CTA at phase boundaries.
-__device__ unsigned long long g_kvp_trace[kPlanGrid][8];
+// [cta][0..7]: phase boundaries; [8]: SM id; [9]: S2 warps done
+__device__ unsigned long long g_kvp_trace[kPlanGrid][12];
 #define KVP_STAMP(i) (g_kvp_trace[blockIdx.x][(i)] = ptx::globaltimer_ns())
 // per-tile events of four CTAs: [cta][tile][event]
 __device__ unsigned long long g_kvp_ttrace[4][64][8];
-__device__ long long g_kvp_mtrace[4][64][12];
+__device__ unsigned long long g_kvp_mtrace[4][64][12];
+#define KVP_MSTAMP(t, e) \
+    ((kvp_trace_slot() >= 0 && (t) < 64) ? (void)(g_kvp_mtrace[kvp_trace_slot()][(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
 __device__ __forceinline__ int kvp_trace_slot() {
     return blockIdx.x == 0 ? 0 : blockIdx.x == 18 ? 1 : blockIdx.x == 73 ? 2 : blockIdx.x == 143 ? 3 : -1;
 }
@@ -82,6 +97,7 @@ __device__ __forceinline__ int kvp_trace_slot() {
 #else
 #define KVP_STAMP(i) ((void)0)
 #define KVP_TSTAMP(t, e) ((void)0)
+#define KVP_MSTAMP(t, e) ((void)0)
 #endif
 
 // error codes recorded in the workspace (first one wins)
@@ -92,8 +108,8 @@ struct Params {
     int nrb, nk0, u0, lg_cpb;  // phase 0: row blocks, keys per unit, units per tile, log2(nk0 / 32)
     int p1, n1, rows16;        // phase 1: parts per tile, rows per part, rows rounded up to 16
     int qrows;                 // query rows staged in shared memory (rows rounded up to 64)
-    int tiles_per_head, total_tiles, grid, cph, maxslots;
-    int ns, nk1, nv1;          // ring slots; phase 1 gives K slots [0, nk1), V slots [nk1, ns)
+    int tiles_per_head, total_tiles, grid, cph, nseg, maxslots;
+    int ns, nk, nv;            // ring slots; phase 1 gives K slots [0, nk), V slots [nk, ns)
     float scale2;              // log2(e) / sqrt(d)
     uint32_t q_bytes, tile_bytes;
     uint32_t off_slots, off_lse, off_comb, off_s2, off_stage, off_wpos, off_bar;
@@ -109,53 +125,58 @@ struct Params {
 
 struct SmemBars {
     uint64_t kfull[kMaxSlots], kempty[kMaxSlots];   // per slot, for its K loads
-    uint64_t vfull[kMaxSlots], vempty[kMaxSlots];   // per phase 1 V slot (index s - nk1)
+    uint64_t vfull[kMaxSlots], vempty[kMaxSlots];   // per phase 1 V slot (index s - nk)
     uint64_t accfull[kStages], accempty[kStages];
     uint64_t combfull[kCombBufs], combempty[kCombBufs];
-    uint64_t s2full[kS2Bufs], s2empty[kS2Bufs];
+    uint64_t s2full[kS2Ring], s2empty[kS2Ring];     // per S2 ring row: its pieces, its readers
+    uint64_t pubfull[2], pubempty[2];               // phase 0 sums of a segment, per buffer
+    uint64_t lsefull[2], lseempty[2];               // phase 1 lse2 of a segment, per buffer
     uint64_t qfull, qempty, fin;
-    uint64_t epi;        // rendezvous of all epilogue threads
     uint32_t tmem_base;
     int abort_flag;
 };
 
 // Wait for phase `parity` of `bar`; false if the CTA is unwinding or the wait timed out
-// (then the first error code is recorded and the CTA told to unwind).
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemBars* sb,
-                                           const Params& p, int code) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+// (then the first error code is recorded and the CTA told to unwind). After the first
+// test the thread sleeps in the barrier (woken by the phase's completion, or after at most
+// kSleepNs to look at the clock), so that waiting warps do not flood shared memory with
+// polls while the TMA, the tensor cores and the working warps use it.
+// The sleeping part is out of line: it is entered only when the first test fails, and
+// one copy of it keeps the kernel's code small.
+constexpr uint32_t kSleepNs = 20000;
+__device__ __noinline__ bool wait_phase_slow(uint64_t* bar, uint32_t parity, int* abort_flag,
+                                             unsigned long long limit_ns, int* err, int code) {
     const uint64_t t0 = ptx::globaltimer_ns();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (ptx::mbar_try_wait(bar, parity)) return true;
-        if (*(volatile int*)&sb->abort_flag) return false;
-        if (ptx::globaltimer_ns() - t0 > p.wait_limit_ns) {
-            atomicCAS(p.err, 0, code);
-            *(volatile int*)&sb->abort_flag = 1;
+        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+        if (*(volatile int*)abort_flag) return false;
+        if (ptx::globaltimer_ns() - t0 > limit_ns) {
+            atomicCAS(err, 0, code);
+            *(volatile int*)abort_flag = 1;
             return false;
         }
     }
+}
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemBars* sb,
+                                           const Params& p, int code) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    return wait_phase_slow(bar, parity, &sb->abort_flag, p.wait_limit_ns, p.err, code);
+}
+
+// wait_phase for the roles whose warps work as a whole (S2, epilogue): the warp takes one
+// decision for all its lanes, so that an abort seen by some lanes only can never split
+// the warp in front of a warp barrier or a warp-collective TMEM load.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, SmemBars* sb,
+                                          const Params& p, int code) {
+    return __all_sync(0xffffffffu, wait_phase(bar, parity, sb, p, code));
 }
 
 // Wait for phase `parity` of `bar` for at most the wait limit, whatever the CTA's state:
 // used before exit, so that no copy or MMA is still writing this CTA's memory.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = ptx::globaltimer_ns();
-    while (!ptx::mbar_try_wait(bar, parity))
+    while (!ptx::mbar_try_wait_sleep(bar, parity, kSleepNs))
         if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) return;
-}
-
-// Rendezvous of all epilogue threads on an mbarrier, so that a thread that gives up a
-// wait can never leave the others blocked in a hardware barrier. One arrival per warp,
-// after the warp's memory writes are ordered before it.
-__device__ __forceinline__ bool epi_sync(SmemBars* sb, uint32_t& phase, const Params& p) {
-    __threadfence_block();
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&sb->epi);
-    const bool ok = wait_phase(&sb->epi, phase, sb, p, kErrWaitEpi);
-    phase ^= 1u;
-    return ok;
 }
 
 __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
@@ -166,20 +187,22 @@ __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
 }
 
 // max |v| over the D bf16 values of one row in shared memory, read in 16-byte pieces in a
-// rotated order per lane (consecutive lanes hit distinct bank groups).
+// rotated order per lane (consecutive lanes hit distinct bank groups), with four
+// independent running maxima so that the reduction is not one long dependent chain.
 template <int D>
 __device__ __forceinline__ float row_absmax(const uint8_t* row, int lane) {
     constexpr int kPieces = D * 2 / 16;
     const uint4* r = reinterpret_cast<const uint4*>(row);
-    uint32_t mx = 0;
-#pragma unroll
+    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll 8
     for (int c = 0; c < kPieces; ++c) {
         const uint4 x = r[(c + lane) & (kPieces - 1)];
-        mx = bf16x2_absmax(mx, x.x & 0x7FFF7FFFu);
-        mx = bf16x2_absmax(mx, x.y & 0x7FFF7FFFu);
-        mx = bf16x2_absmax(mx, x.z & 0x7FFF7FFFu);
-        mx = bf16x2_absmax(mx, x.w & 0x7FFF7FFFu);
+        m0 = bf16x2_absmax(m0, x.x & 0x7FFF7FFFu);
+        m1 = bf16x2_absmax(m1, x.y & 0x7FFF7FFFu);
+        m2 = bf16x2_absmax(m2, x.z & 0x7FFF7FFFu);
+        m3 = bf16x2_absmax(m3, x.w & 0x7FFF7FFFu);
     }
+    const uint32_t mx = bf16x2_absmax(bf16x2_absmax(m0, m1), bf16x2_absmax(m2, m3));
     return fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
 }
 
@@ -188,28 +211,37 @@ __device__ __forceinline__ int ring_uses(int s, int period, int n) {
     return n > s ? (n - s + period - 1) / period : 0;
 }
 // K slot of the run's tile i in `phase`, and the number of that slot's earlier K loads.
-// Phase 0 streams K through all ns slots in turn; phase 1 through slots [0, nk1).
+// Phase 0 streams K through all ns slots in turn; phase 1 through slots [0, nk).
 __device__ __forceinline__ int k_slot(int phase, int i, int n, const Params& p, int& use) {
     if (phase == 0) {
         use = i / p.ns;
         return i % p.ns;
     }
-    const int s = i % p.nk1;
-    use = ring_uses(s, p.ns, n) + i / p.nk1;
+    const int s = i % p.nk;
+    use = ring_uses(s, p.ns, n) + i / p.nk;
     return s;
 }
 
-// Segments of a CTA's run: maximal stretches of tiles within one KV head.
-struct RunIter {
-    long long t, end;
-    int tph;
-    __device__ RunIter(long long b, long long e, int tiles_per_head) : t(b), end(e), tph(tiles_per_head) {}
-    __device__ bool next(int& head, long long& a, long long& b) {
-        if (t >= end) return false;
-        head = (int)(t / tph);
+// The CTA's work in one phase: its segments in order, each split where it crosses a KV
+// head (only flat runs do), with the slot of the CTA's partial in that head.
+// Tile numbers fit in 32 bits (the plan checks it).
+struct CtaRun {
+    const Params* p;
+    int s, t, end;
+    __device__ explicit CtaRun(const Params& prm) : p(&prm), s(-1), t(0), end(0) {}
+    __device__ bool next(int& head, int& a, int& b, int& slot) {
+        while (t >= end) {
+            if (++s >= p->nseg) return false;
+            uint32_t tb, te;
+            segment_of_u32(blockIdx.x, s, p->total_tiles, p->grid, p->tiles_per_head, p->cph, tb, te);
+            t = (int)tb;
+            end = (int)te;
+        }
+        head = t / p->tiles_per_head;
         a = t;
-        b = min(end, (long long)(head + 1) * tph);
+        b = min(end, (head + 1) * p->tiles_per_head);
         t = b;
+        slot = (int)slot_in_head_u32(blockIdx.x, s, head, p->total_tiles, p->grid, p->tiles_per_head, p->cph);
         return true;
     }
 };
@@ -298,6 +330,45 @@ __device__ __forceinline__ float s1_chunk(const float (&v)[32], const float* lse
     return (a0 + a1) + (a2 + a3);
 }
 
+// Phase 1's V stream for a warp of its own (two such warps share it): take the next piece
+// (32 keys of a tile) by ticket, wait until its tile has landed and its S2 ring row is
+// free, reduce each key to S2 = max |V| (one key per lane) into the ring, and release the
+// piece's share of the V slot and of the ring row. A worker only ever waits on the barriers
+// of a piece it holds, whose phases cannot move on before it is done. Every wait sleeps in
+// the barrier and is bounded.
+template <int D>
+__device__ __forceinline__ void v_worker(uint8_t* smem, const Params& p, int n, SmemBars* sb) {
+    constexpr uint32_t kSlotBytes = kTile * D * 2;
+    constexpr int kKeys = kTile / kVPieces;               // keys per piece: one per lane
+    static_assert(kKeys == 32, "one key per lane");
+    const int lane = threadIdx.x & 31;
+    const uint8_t* Slots = smem + p.off_slots;
+    float* s2ring = (float*)(smem + p.off_s2);
+    uint32_t* vclaim = (uint32_t*)(s2ring + kS2Ring * kTile);
+    const uint32_t npieces = (uint32_t)(kVPieces * n);
+    while (true) {
+        uint32_t c = 0;
+        if (lane == 0) c = atomicAdd(vclaim, 1u);
+        c = __shfl_sync(0xffffffffu, c, 0);
+        if (c >= npieces) break;
+        const int vi = (int)(c / kVPieces), rs = vi & (kS2Ring - 1);
+        if (vi >= kS2Ring && !wait_warp(&sb->s2empty[rs], (vi / kS2Ring - 1) & 1, sb, p, kErrWaitS2)) break;
+        if (!wait_warp(&sb->vfull[vi % p.nv], (vi / p.nv) & 1, sb, p, kErrWaitS2)) break;
+        if (lane == 0 && c % kVPieces == 0) KVP_MSTAMP(vi, 0);
+        const int key = (int)(c % kVPieces) * kKeys + lane;
+        const float s2 = row_absmax<D>(Slots + (p.nk + vi % p.nv) * kSlotBytes + key * (D * 2), lane);
+        __syncwarp();                                     // every lane is done with the V slot
+        if (lane == 0) ptx::mbar_arrive(&sb->vempty[vi % p.nv]);
+        s2ring[rs * kTile + key] = s2;
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            ptx::mbar_arrive(&sb->s2full[rs]);
+            if (c % kVPieces == kVPieces - 1) KVP_MSTAMP(vi, 1);
+        }
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -306,10 +377,11 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* Qs = smem;                                  // [D / 64][qrows][64] bf16, 128B swizzle
     uint8_t* Slots = smem + p.off_slots;                 // ring slots of tile_bytes each
-    float* lse2 = (float*)(smem + p.off_lse);            // [rows, padded to 4]
-    float* comb = (float*)(smem + p.off_comb);           // [kCombBufs][128] partial S1 hand-off
-    float* s2buf = (float*)(smem + p.off_s2);            // [kS2Bufs][128] S2 of a tile's keys
-    float2* stage0 = (float2*)(smem + p.off_stage);      // [rows] phase 0 group hand-off
+    float* lse2 = (float*)(smem + p.off_lse);            // [2][rows4]: a segment's lse2 per buffer
+    float* comb = (float*)(smem + p.off_comb);           // [kCombBufs][kMaxParts - 1][128]
+    float2* pub = (float2*)(smem + p.off_stage);         // [2][kGroups][rows] phase 0 (m, l)
+    float* s2ring = (float*)(smem + p.off_s2);           // [kS2Ring][128] S2 of a tile's keys
+    uint32_t* vclaim = (uint32_t*)(s2ring + kS2Ring * kTile);  // V piece tickets taken
     uint16_t* wpos = (uint16_t*)(smem + p.off_wpos);     // window position of query row n: n % w
     SmemBars* sb = (SmemBars*)(smem + p.off_bar);
 
@@ -317,38 +389,47 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     constexpr uint32_t kHalfTile = kTile * 128;     // bytes of one 64-column half of a tile
     constexpr uint32_t kSlotBytes = kTile * D * 2;
     const uint32_t qhalf = (uint32_t)p.qrows * 128;  // bytes of one 64-column half of Q
+    const int rows4 = (p.rows + 3) & ~3;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long T = p.total_tiles;
-    const long long t0 = run_begin(blockIdx.x, T, p.grid, p.tiles_per_head, p.cph);
-    const long long t1 = run_begin(blockIdx.x + 1, T, p.grid, p.tiles_per_head, p.cph);
-    const int n = (int)(t1 - t0);                   // tiles in this CTA's run
+    int n = 0;                                      // tiles in this CTA's run
+    for (int s = 0; s < p.nseg; ++s) {
+        uint32_t b, e;
+        segment_of_u32(blockIdx.x, s, p.total_tiles, p.grid, p.tiles_per_head, p.cph, b, e);
+        n += (int)(e - b);
+    }
     const int U0 = n * p.u0;                        // phase 0 units of the run
 
     for (int r = threadIdx.x; r < p.rows; r += kThreads) wpos[r] = (uint16_t)(r % p.w);
+    if (threadIdx.x == 0) *vclaim = 0u;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxSlots; ++s) {
             ptx::mbar_init(&sb->kfull[s], 1);
             ptx::mbar_init(&sb->kempty[s], 1);
             ptx::mbar_init(&sb->vfull[s], 1);
-            ptx::mbar_init(&sb->vempty[s], kS2Warps);
+            ptx::mbar_init(&sb->vempty[s], kVPieces);
         }
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(&sb->accfull[s], 1);
             ptx::mbar_init(&sb->accempty[s], 4);
         }
+        for (int s = 0; s < kS2Ring; ++s) {
+            ptx::mbar_init(&sb->s2full[s], kVPieces);
+            ptx::mbar_init(&sb->s2empty[s], 4);        // the finishing group's four warps
+        }
         for (int s = 0; s < kCombBufs; ++s) {
-            ptx::mbar_init(&sb->combfull[s], 4);
+            ptx::mbar_init(&sb->combfull[s], 4 * (p.p1 - 1 > 0 ? p.p1 - 1 : 1));
             ptx::mbar_init(&sb->combempty[s], 4);
         }
-        for (int s = 0; s < kS2Bufs; ++s) {
-            ptx::mbar_init(&sb->s2full[s], kS2Warps);
-            ptx::mbar_init(&sb->s2empty[s], 4);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&sb->pubfull[s], kEpiThreads / 32);
+            ptx::mbar_init(&sb->pubempty[s], 1);
+            ptx::mbar_init(&sb->lsefull[s], kEpiThreads / 32);
+            ptx::mbar_init(&sb->lseempty[s], kEpiThreads / 32);
         }
         ptx::mbar_init(&sb->qfull, 1);
         ptx::mbar_init(&sb->qempty, 1);
         ptx::mbar_init(&sb->fin, 1);
-        ptx::mbar_init(&sb->epi, kEpiThreads / 32);
         sb->abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -366,73 +447,82 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     ptx::tc_fence_after();
     const uint32_t tmem = sb->tmem_base;
     if (threadIdx.x == 0) KVP_STAMP(0);
+#ifdef KVP_TRACE
+    if (threadIdx.x == 0) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        g_kvp_trace[blockIdx.x][8] = smid;
+    }
+#endif
 
     auto group_row0 = [&](int bh) {
         const int b = bh / p.hkv, h = bh % p.hkv;
         return (b * p.hq + h * p.G) * p.w;
     };
 
+
+    // Roles are dispatched on whole warps: every lane of a warp takes the same branch, and a
+    // single-lane role sits inside its warp's branch, so no lane can fall into another role.
     if (warp == 0) {
+      if (lane == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            // K is read again by phase 1 (from L2 when it fits); V and phase 1's K stream
-            const uint64_t pol_keep = ptx::policy_evict_normal();
-            const uint64_t pol_stream = ptx::policy_evict_first();
-            int qgen = 0, cur = -1;
-            int kiss[kMaxSlots] = {}, viss[kMaxSlots] = {};   // loads issued per slot
-            bool ok = true;
-            for (int phase = 0; phase < 2 && ok; ++phase) {
-                RunIter it(t0, t1, p.tiles_per_head);
-                int head;
-                long long a, b;
-                int i = 0;                                  // tile number within the run
-                while (ok && it.next(head, a, b)) {
-                    if (head != cur) {
-                        if (qgen > 0 && !(ok = wait_phase(&sb->qempty, (qgen - 1) & 1, sb, p, kErrWaitTma))) break;
-                        ptx::mbar_arrive_expect_tx(&sb->qfull, p.q_bytes);
-                        const int r0 = group_row0(head);
-                        for (int rb = 0; rb < p.qrows; rb += kQBoxRows)
-                            for (int c = 0; c < kHalves; ++c)
-                                ptx::tma_load_2d(Qs + c * qhalf + rb * 128, &qmap, &sb->qfull,
-                                                 c * 64, r0 + rb, pol_keep);
-                        ++qgen;
-                        cur = head;
-                    }
-                    for (long long t = a; t < b; ++t, ++i) {
-                        const int key0 = (int)(t - (long long)head * p.tiles_per_head) * kTile;
-                        int use;
-                        const int s = k_slot(phase, i, n, p, use);
-                        if (!(ok = wait_phase(&sb->kempty[s], (use & 1) ^ 1, sb, p, kErrWaitTma))) break;
-                        KVP_TSTAMP(phase * n + i, 0);
-                        ptx::mbar_arrive_expect_tx(&sb->kfull[s], p.tile_bytes);
+        // K is read again by phase 1 (from L2 when it fits); V and phase 1's K stream
+        const uint64_t pol_keep = ptx::policy_evict_normal();
+        const uint64_t pol_stream = ptx::policy_evict_first();
+        int qgen = 0, cur = -1;
+        int kiss[kMaxSlots] = {}, viss[kMaxSlots] = {};     // loads issued per slot
+        bool ok = true;
+        for (int phase = 0; phase < 2 && ok; ++phase) {
+            CtaRun it(p);
+            int head, slot, a, b;
+            int i = 0;                                      // tile number within the run
+            while (ok && it.next(head, a, b, slot)) {
+                if (head != cur) {
+                    if (qgen > 0 && !(ok = wait_phase(&sb->qempty, (qgen - 1) & 1, sb, p, kErrWaitTma))) break;
+                    ptx::mbar_arrive_expect_tx(&sb->qfull, p.q_bytes);
+                    const int r0 = group_row0(head);
+                    for (int rb = 0; rb < p.qrows; rb += kQBoxRows)
                         for (int c = 0; c < kHalves; ++c)
-                            ptx::tma_load_3d(Slots + s * kSlotBytes + c * kHalfTile, &kmap, &sb->kfull[s],
-                                             c * 64, key0, head, phase == 0 ? pol_keep : pol_stream);
-                        ++kiss[s];
-                        if (phase == 1) {
-                            const int jv = i % p.nv1, sv = p.nk1 + jv, vuse = i / p.nv1;
-                            // a V slot's first load waits for its last K load of phase 0 to be consumed
-                            const int u0s = vuse == 0 ? ring_uses(sv, p.ns, n) : 0;
-                            if (u0s > 0 && !(ok = wait_phase(&sb->kempty[sv], (u0s - 1) & 1, sb, p, kErrWaitTma))) break;
-                            if (!(ok = wait_phase(&sb->vempty[jv], (vuse & 1) ^ 1, sb, p, kErrWaitTma))) break;
-                            KVP_TSTAMP(phase * n + i, 6);
-                            ptx::mbar_arrive_expect_tx(&sb->vfull[jv], p.tile_bytes);
-                            ptx::tma_load_3d(Slots + sv * kSlotBytes, &vmap, &sb->vfull[jv], 0, key0, head,
-                                             pol_stream);
-                            ++viss[jv];
-                        }
+                            ptx::tma_load_2d(Qs + c * qhalf + rb * 128, &qmap, &sb->qfull,
+                                             c * 64, r0 + rb, pol_keep);
+                    ++qgen;
+                    cur = head;
+                }
+                for (int t = a; t < b; ++t, ++i) {
+                    const int key0 = (t - head * p.tiles_per_head) * kTile;
+                    int use;
+                    const int s = k_slot(phase, i, n, p, use);
+                    if (!(ok = wait_phase(&sb->kempty[s], (use & 1) ^ 1, sb, p, kErrWaitTma))) break;
+                    KVP_TSTAMP(phase * n + i, 0);
+                    ptx::mbar_arrive_expect_tx(&sb->kfull[s], p.tile_bytes);
+                    for (int c = 0; c < kHalves; ++c)
+                        ptx::tma_load_3d(Slots + s * kSlotBytes + c * kHalfTile, &kmap, &sb->kfull[s],
+                                         c * 64, key0, head, phase == 0 ? pol_keep : pol_stream);
+                    ++kiss[s];
+                    if (phase == 1) {
+                        const int jv = i % p.nv, sv = p.nk + jv, vuse = i / p.nv;
+                        // a V slot's first load waits for its last K load of phase 0 to be consumed
+                        const int u0s = vuse == 0 ? ring_uses(sv, p.ns, n) : 0;
+                        if (u0s > 0 && !(ok = wait_phase(&sb->kempty[sv], (u0s - 1) & 1, sb, p, kErrWaitTma))) break;
+                        if (!(ok = wait_phase(&sb->vempty[jv], (vuse & 1) ^ 1, sb, p, kErrWaitTma))) break;
+                        KVP_TSTAMP(n + i, 6);
+                        ptx::mbar_arrive_expect_tx(&sb->vfull[jv], p.tile_bytes);
+                        ptx::tma_load_3d(Slots + sv * kSlotBytes, &vmap, &sb->vfull[jv], 0, key0, head,
+                                         pol_stream);
+                        ++viss[jv];
                     }
                 }
-                KVP_STAMP(1 + phase);
             }
-            // Never leave with copies in flight: wait for the last load issued to every slot
-            // (these waits do not stop early when the CTA unwinds).
-            for (int s = 0; s < p.ns; ++s)
-                if (kiss[s] > 0) drain_wait(&sb->kfull[s], (kiss[s] - 1) & 1);
-            for (int jv = 0; jv < p.nv1; ++jv)
-                if (viss[jv] > 0) drain_wait(&sb->vfull[jv], (viss[jv] - 1) & 1);
-            if (qgen > 0) drain_wait(&sb->qfull, (qgen - 1) & 1);
+            KVP_STAMP(1 + phase);
         }
+        // Never leave with copies in flight: wait for the last load issued to every slot
+        // (these waits do not stop early when the CTA unwinds).
+        for (int s = 0; s < p.ns; ++s)
+            if (kiss[s] > 0) drain_wait(&sb->kfull[s], (kiss[s] - 1) & 1);
+        for (int jv = 0; jv < p.nv; ++jv)
+            if (viss[jv] > 0) drain_wait(&sb->vfull[jv], (viss[jv] - 1) & 1);
+        if (qgen > 0) drain_wait(&sb->qfull, (qgen - 1) & 1);
+      }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -441,19 +531,18 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             int qgen = 0, cur = -1;
             bool ok = true;
             for (int phase = 0; phase < 2 && ok; ++phase) {
-                RunIter it(t0, t1, p.tiles_per_head);
-                int head;
-                long long a, b;
+                CtaRun it(p);
+                int head, slot, a, b;
                 int i = 0;                                  // tile number within the run
                 int unit = 0;                               // unit number within the phase
-                while (ok && it.next(head, a, b)) {
+                while (ok && it.next(head, a, b, slot)) {
                     if (head != cur) {
                         if (!(ok = wait_phase(&sb->qfull, qgen & 1, sb, p, kErrWaitMma))) break;
                         ++qgen;
                         cur = head;
                         ptx::tc_fence_after();
                     }
-                    for (long long t = a; t < b && ok; ++t, ++i) {
+                    for (int t = a; t < b && ok; ++t, ++i) {
                         int kuse;
                         const int s = k_slot(phase, i, n, p, kuse);
                         if (!(ok = wait_phase(&sb->kfull[s], kuse & 1, sb, p, kErrWaitMma))) break;
@@ -464,6 +553,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                             const int st = unit & (kStages - 1);
                             const int use = (phase == 0 ? 0 : ring_uses(st, kStages, U0)) + unit / kStages;
                             if (!(ok = wait_phase(&sb->accempty[st], (use & 1) ^ 1, sb, p, kErrWaitMma))) break;
+                            if (j == 0) KVP_TSTAMP(phase * n + i, 2);
                             ptx::tc_fence_after();
                             const uint32_t d0 = tmem + (uint32_t)(st * kStageCols);
                             if (phase == 0) {
@@ -500,13 +590,12 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     if (!ok) break;
                     // release the query rows when the next segment loads another head's
                     {
-                        RunIter peek = it;
-                        int nh = -1;
-                        long long na, nb;
-                        bool more = peek.next(nh, na, nb);
+                        CtaRun peek = it;
+                        int nh = -1, ns2, na, nb;
+                        bool more = peek.next(nh, na, nb, ns2);
                         if (!more && phase == 0) {
-                            RunIter again(t0, t1, p.tiles_per_head);
-                            more = again.next(nh, na, nb);
+                            CtaRun again(p);
+                            more = again.next(nh, na, nb, ns2);
                         }
                         if (more && nh != cur) ptx::mma_commit(&sb->qempty);
                     }
@@ -518,71 +607,93 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             ptx::mma_commit(&sb->fin);
             drain_wait(&sb->fin, 0);
         }
-    } else if (warp < kWarpEpi) {
-        // ------------------------------------------------------------ S2: max |V| per key
-        const int k2 = threadIdx.x - 32 * kWarpS2;          // 0 .. 63: keys k2 and k2 + 64
+    } else if (warp == kWarpPub) {
+        // ------------------------------------------------------------ phase 0 publisher
+        // Per segment: combine the epilogue groups' (m, l) of every row, write the CTA's
+        // slot, then bump the head's completion counter (so that no epilogue thread waits on
+        // a global fence).
         bool ok = true;
-        for (int i = 0; i < n && ok; ++i) {
-            const int jv = i % p.nv1, vuse = i / p.nv1;
-            if (!(ok = wait_phase(&sb->vfull[jv], vuse & 1, sb, p, kErrWaitS2))) break;
-            const uint8_t* vt = Slots + (p.nk1 + jv) * kSlotBytes;
-            const float ra = row_absmax<D>(vt + k2 * (D * 2), lane);
-            const float rb = row_absmax<D>(vt + (k2 + 64) * (D * 2), lane);
+        CtaRun it(p);
+        int head, slot, a, b;
+        int k = 0;
+        while (ok && it.next(head, a, b, slot)) {
+            const int buf = k & 1, use = k >> 1;
+            if (!(ok = wait_warp(&sb->pubfull[buf], use & 1, sb, p, kErrWaitEpi))) break;
+            const int r0 = group_row0(head);
+            const float2* pbuf = pub + (size_t)buf * kGroups * p.rows;
+            for (int r = lane; r < p.rows; r += 32) {
+                float2 o[kGroups];
+                float M = -INFINITY;
+#pragma unroll
+                for (int g = 0; g < kGroups; ++g) {
+                    o[g] = pbuf[g * p.rows + r];
+                    M = fmaxf(M, o[g].x);
+                }
+                float S = 0.f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int g = 0; g < kGroups; ++g) S += o[g].y * ptx::ex2(o[g].x - M);
+                }
+                if (KVP_CHECK(slot >= 0 && slot < p.maxslots, 202, slot, head))
+                    p.part[(size_t)(r0 + r) * p.maxslots + slot] = make_float2(M, S);
+            }
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&sb->vempty[jv]);
-            const int e = i & (kS2Bufs - 1), use = i / kS2Bufs;
-            if (!(ok = wait_phase(&sb->s2empty[e], (use & 1) ^ 1, sb, p, kErrWaitS2))) break;
-            s2buf[e * kTile + k2] = ra;
-            s2buf[e * kTile + k2 + 64] = rb;
+            if (lane == 0) ptx::mbar_arrive(&sb->pubempty[buf]);
+            __threadfence();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&sb->s2full[e]);
+            if (lane == 0) atomicAdd(p.done + head, 1u);
+            ++k;
         }
-    } else {
-        // ------------------------------------------------------------ epilogue
+        if (lane == 0) KVP_STAMP(5);
+        if (ok) v_worker<D>(smem, p, n, sb);
+    } else if (warp == kWarpV) {
+        // ------------------------------------------------------------ V pieces
+        v_worker<D>(smem, p, n, sb);
+    } else if (warp >= kWarpEpi) {
+        // ------------------------------------------------------------ epilogue (warps 4-19)
         const int et = threadIdx.x - 32 * kWarpEpi;      // 0 .. kEpiThreads-1
-        const int eg = et >> 7;                           // epilogue group
+        const int eg = et >> 7;                           // epilogue group = its TMEM stage
         const int quarter = warp & 3;                     // TMEM lane quarter of this warp
         const int lq = quarter * 32 + lane;               // lane: query row (phase 0) / key (phase 1)
         const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t tst = tlane + (uint32_t)(eg * kStageCols);
         const int window0 = p.L - p.w;                    // first window position
-        uint32_t epi_phase = 0;
         bool ok = true;
         // ---- phase 0: per query row, the running offset and sum of 2^(t - m) over the keys
         //      of this group's units (thread = row, TMEM columns = keys)
         {
-            // last visible key of this thread's row in each row block
-            int lim[4];
-#pragma unroll
-            for (int rb = 0; rb < 4; ++rb) lim[rb] = window0 + (rb * 128 + lq) % p.w;
-            // chunks of a unit that hold rows of this warp: all rows of a row block
-            // are live or none, and live chunks are a prefix of the unit's four
+            // chunks of a unit that hold rows of this warp: all rows of a row block are live
+            // or none, and live chunks are a prefix of the unit's four
             const int rbl = p.rows > quarter * 32 ? min(p.nrb, (p.rows - quarter * 32 + 127) / 128) : 0;
             const int nl = min(4, rbl << p.lg_cpb);
             const int cmask = (1 << p.lg_cpb) - 1;
-            RunIter it(t0, t1, p.tiles_per_head);
-            int head;
-            long long a, b;
-            int unit = 0, i = 0;
-            while (ok && it.next(head, a, b)) {
+            CtaRun it(p);
+            int head, slot, a, b;
+            int unit = 0, i = 0, k = 0;
+            while (ok && it.next(head, a, b, slot)) {
                 float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 float l[4] = {0.f, 0.f, 0.f, 0.f};
-                for (long long t = a; t < b && ok; ++t, ++i) {
-                    const int key_t = (int)(t - (long long)head * p.tiles_per_head) * kTile;
+                for (int t = a; t < b && ok; ++t, ++i) {
+                    const int key_t = (t - head * p.tiles_per_head) * kTile;
                     for (int j = 0; j < p.u0; ++j, ++unit) {
-                        if ((unit & 1) != eg) continue;      // the other group's unit
-                        const int st = unit & (kStages - 1);
-                        if (!(ok = wait_phase(&sb->accfull[st], (unit / kStages) & 1, sb, p, kErrWaitEpi))) break;
+                        if ((unit & (kStages - 1)) != eg) continue;   // another group's unit
+                        if (!(ok = wait_warp(&sb->accfull[eg], (unit / kStages) & 1, sb, p, kErrWaitEpi))) break;
                         if (lq == 0) KVP_TSTAMP(i, 4);
                         ptx::tc_fence_after();
                         const int kbase = key_t + j * p.nk0;
-                        const uint32_t tst = tlane + (uint32_t)(st * kStageCols);
                         // chunk c: TMEM columns [32c, 32c + 32) of the stage, row block c >> lg_cpb,
                         // keys kbase + 32 (c & cmask) + e
-                        auto proc = [&](float (&v)[32], int c) {
+#pragma unroll 1
+                        for (int c = 0; c < nl; ++c) {
+                            float v[32];
+                            __syncwarp();
+                            ptx::tmem_ld_32x32b_x32(tst + c * 32, v);
+                            ptx::tmem_ld_wait(v);
                             const int rb = c >> p.lg_cpb;
                             const int j0 = kbase + ((c & cmask) << 5);
                             if (j0 + 31 > window0) {         // window or ragged keys: mask per row
-                                const int rel = pick4(lim, rb) - j0;
+                                // the row's last visible key is window0 + its window position
+                                const int rel = window0 + (rb * 128 + lq) % p.w - j0;
 #pragma unroll
                                 for (int e = 0; e < 32; ++e)
                                     if (e > rel) v[e] = -INFINITY;
@@ -591,209 +702,174 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                             lse_chunk(v, p.scale2, mr, lr);
                             put4(m, rb, mr);
                             put4(l, rb, lr);
-                        };
-                        if (nl > 0) {
-                            float x[32], y[32];
-                            __syncwarp();
-                            ptx::tmem_ld_32x32b_x32(tst, x);
-                            ptx::tmem_ld_wait(x);
-#pragma unroll 1
-                            for (int c = 0; c < nl; c += 2) {
-                                const bool h1 = c + 1 < nl, h2 = c + 2 < nl;
-                                if (h1) {
-                                    __syncwarp();
-                                    ptx::tmem_ld_32x32b_x32(tst + (c + 1) * 32, y);
-                                }
-                                proc(x, c);
-                                if (h1) {
-                                    ptx::tmem_ld_wait(y);
-                                    if (h2) {
-                                        __syncwarp();
-                                        ptx::tmem_ld_32x32b_x32(tst + (c + 2) * 32, x);
-                                    }
-                                    proc(y, c + 1);
-                                    if (h2) ptx::tmem_ld_wait(x);
-                                }
-                            }
                         }
                         ptx::tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&sb->accempty[st]);
+                        if (lane == 0) ptx::mbar_arrive(&sb->accempty[eg]);
                         if (lq == 0) KVP_TSTAMP(i, 5);
                     }
                 }
                 if (!ok) break;
-                // Combine the two groups' (m, l) of every row, then publish one slot per row.
-                if (!(ok = epi_sync(sb, epi_phase, p))) break;   // stage0 free again
-                if (eg == 1) {
+                // hand this group's (m, l) of every row to the publisher and go on
+                const int buf = k & 1, use = k >> 1;
+                if (!(ok = wait_warp(&sb->pubempty[buf], (use & 1) ^ 1, sb, p, kErrWaitEpi))) break;
+                float2* pb = pub + ((size_t)buf * kGroups + eg) * p.rows;
 #pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        const int r = rb * 128 + lq;
-                        if (rb < p.nrb && r < p.rows) stage0[r] = make_float2(m[rb], l[rb]);
-                    }
+                for (int rb = 0; rb < 4; ++rb) {
+                    const int r = rb * 128 + lq;
+                    if (rb < p.nrb && r < p.rows) pb[r] = make_float2(m[rb], l[rb]);
                 }
-                if (!(ok = epi_sync(sb, epi_phase, p))) break;
-                if (eg == 0) {
-                    const long long first = (long long)head * p.tiles_per_head;
-                    const int slot = (int)blockIdx.x - owner_of(first, T, p.grid, p.tiles_per_head, p.cph);
-                    const int r0 = group_row0(head);
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        const int r = rb * 128 + lq;
-                        if (rb < p.nrb && r < p.rows) {
-                            const float2 o = stage0[r];
-                            const float M = fmaxf(m[rb], o.x);
-                            float S = 0.f;
-                            if (M != -INFINITY) S = l[rb] * ptx::ex2(m[rb] - M) + o.y * ptx::ex2(o.x - M);
-                            if (KVP_CHECK(slot >= 0 && slot < p.maxslots, 202, slot, head))
-                                p.part[(size_t)(r0 + r) * p.maxslots + slot] = make_float2(M, S);
-                        }
-                    }
-                    __threadfence();
-                }
-                if (!(ok = epi_sync(sb, epi_phase, p))) break;
-                if (et == 0) {
-                    __threadfence();
-                    atomicAdd(p.done + head, 1u);
-                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sb->pubfull[buf]);
+                ++k;
             }
         }
-        if (et == 0) KVP_STAMP(5);
+        // Wait for `cond` (a warp-uniform test of memory that no barrier guards), polling;
+        // bounded.
+        auto pwait = [&](auto&& cond, int code) -> bool {
+            if (cond()) return true;
+            // the low 32 bits of the ns timer: they wrap every 4.29 s, above any wait limit
+            const uint32_t t0 = (uint32_t)ptx::globaltimer_ns();
+            while (true) {
+                __nanosleep(256);
+                if (cond()) return true;
+                if (__any_sync(0xffffffffu, *(volatile int*)&sb->abort_flag != 0)) return false;
+                // one decision for the warp: its lanes read the clock at slightly different times
+                if (__any_sync(0xffffffffu, (uint32_t)ptx::globaltimer_ns() - t0 > (uint32_t)p.wait_limit_ns)) {
+                    if (lane == 0) {
+                        atomicCAS(p.err, 0, code);
+                        *(volatile int*)&sb->abort_flag = 1;
+                    }
+                    return false;
+                }
+            }
+        };
+        auto bwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return wait_warp(bar, parity, sb, p, kErrWaitEpi);
+        };
         // ---- phase 1: scores (thread = key, TMEM columns = query rows)
         {
             bool first_seg = true;
-            RunIter it(t0, t1, p.tiles_per_head);
-            int head;
-            long long a, b;
-            int unit = 0, i = 0;
-            while (ok && it.next(head, a, b)) {
-                const long long first = (long long)head * p.tiles_per_head;
-                const int touch = owner_of(first + p.tiles_per_head - 1, T, p.grid, p.tiles_per_head, p.cph) -
-                                  owner_of(first, T, p.grid, p.tiles_per_head, p.cph) + 1 + p.extra_peers;
-                // the previous head's lse2 is no longer in use
-                if (!(ok = epi_sync(sb, epi_phase, p))) break;
-                if (et == 0) {
-                    const uint64_t ts = ptx::globaltimer_ns();
-                    while (ptx::ld_acquire_u32(p.done + head) < (uint32_t)touch) {
-                        if (*(volatile int*)&sb->abort_flag) break;
-                        if (ptx::globaltimer_ns() - ts > p.wait_limit_ns) {
-                            atomicCAS(p.err, 0, kErrWaitPeers);
-                            *(volatile int*)&sb->abort_flag = 1;
-                            break;
-                        }
-                        __nanosleep(128);
-                    }
-                }
-                if (!(ok = epi_sync(sb, epi_phase, p))) break;
+            CtaRun it(p);
+            int head, slot, a, b;
+            int i = 0, k = 0;
+            while (ok && it.next(head, a, b, slot)) {
+                const int first = head * p.tiles_per_head;
+                const int buf = k & 1, use = k >> 1;
+                float* ls = lse2 + buf * rows4;
+                // This group merges the head's slots into lse2 for its share of the rows (the
+                // 32-row blocks b with b % 4 == eg), once the buffer is free and every CTA
+                // touching the head has published.
+                if (!(ok = bwait(&sb->lseempty[buf], (use & 1) ^ 1))) break;
+                const int touch = (int)ctas_touching_u32(head, p.total_tiles, p.grid, p.tiles_per_head, p.cph);
+                const uint32_t want = (uint32_t)(touch + p.extra_peers);
+                if (!(ok = pwait([&]() {
+                          uint32_t d = 0;
+                          if (lane == 0) d = ptx::ld_acquire_u32(p.done + head);
+                          return __shfl_sync(0xffffffffu, d, 0) >= want;
+                      }, kErrWaitPeers)))
+                    break;
+                (void)ptx::ld_acquire_u32(p.done + head);     // every lane acquires the slots
                 if (et == 0 && first_seg) KVP_STAMP(6);
                 first_seg = false;
-                if (*(volatile int*)&sb->abort_flag) {
-                    ok = false;
-                    break;
-                }
                 const int r0 = group_row0(head);
-                const int nslots = (touch - p.extra_peers) * kSlotsPerCta;
-                // Two threads per row, each over every other slot: first the row's
-                // maximum, then the sum of l 2^(m - max); every load and term independent.
-                for (int base = 0; base < 2 * p.rows; base += kEpiThreads) {
-                    const int r2 = base + et, r = r2 >> 1;
-                    const float2* pr = p.part + (size_t)(r0 + (r < p.rows ? r : 0)) * p.maxslots;
-                    float M = -INFINITY;
+                const int nslots = touch * kSlotsPerCta;
+                // four threads per row, each over every fourth slot, in one pass (a running
+                // maximum with the sum rescaled when it rises)
+                for (int rr = (et & 127) >> 2; ; rr += 32) {
+                    const int r = ((rr >> 5) * kGroups + eg) * 32 + (rr & 31);
+                    if (__all_sync(0xffffffffu, r >= p.rows)) break;
+                    const int q = et & 3;
+                    float M = -INFINITY, S = 0.f;
                     if (r < p.rows) {
+                        const float2* pr = p.part + (size_t)(r0 + r) * p.maxslots;
 #pragma unroll 4
-                        for (int sl = r2 & 1; sl < nslots; sl += 2) {
+                        for (int sl = q; sl < nslots; sl += 4) {
                             const float2 ml = __ldcg(pr + sl);
-                            if (ml.y != 0.f) M = fmaxf(M, ml.x);
+                            if (ml.y != 0.f) {
+                                if (ml.x > M) {
+                                    S = S * ptx::ex2(M - ml.x) + ml.y;
+                                    M = ml.x;
+                                } else {
+                                    S += ml.y * ptx::ex2(ml.x - M);
+                                }
+                            }
                         }
                     }
-                    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
-                    float S = 0.f;
-                    if (r < p.rows && M != -INFINITY) {
-#pragma unroll 4
-                        for (int sl = r2 & 1; sl < nslots; sl += 2) {
-                            const float2 ml = __ldcg(pr + sl);
-                            if (ml.y != 0.f) S += ml.y * ptx::ex2(ml.x - M);
-                        }
+#pragma unroll
+                    for (int o = 1; o <= 2; o <<= 1) {
+                        const float Mo = __shfl_xor_sync(0xffffffffu, M, o);
+                        const float So = __shfl_xor_sync(0xffffffffu, S, o);
+                        const float Mn = fmaxf(M, Mo);
+                        S = (Mn == -INFINITY) ? 0.f : S * ptx::ex2(M - Mn) + So * ptx::ex2(Mo - Mn);
+                        M = Mn;
                     }
-                    S += __shfl_xor_sync(0xffffffffu, S, 1);
-                    if (r < p.rows && (r2 & 1) == 0) lse2[r] = M + __log2f(S);
+                    if (r < p.rows && q == 0) ls[r] = M + __log2f(S);
                 }
-                if (!(ok = epi_sync(sb, epi_phase, p))) break;
-                for (long long t = a; t < b && ok; ++t, ++i) {
-                    const int j = (int)(t - first) * kTile + lq;     // this thread's key
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sb->lsefull[buf]);
+                if (!(ok = bwait(&sb->lsefull[buf], use & 1))) break;
+                for (int t = a; t < b && ok; ++t, ++i) {
+                    const int j = (t - first) * kTile + lq;          // this thread's key
                     const int jw = j - window0;                      // > 0 only inside the window
+                    // units of this tile: i * p1 + part, in stages (and groups) (i * p1 + part) % 4
+                    const int u_first = i * p.p1;
+                    const int pp = (eg - u_first) & (kStages - 1);   // this group's part, if any
+                    if (pp >= p.p1) continue;                        // not this group's tile
+                    const int myunit = u_first + pp;
                     // masks (window keys) are decided per warp: TMEM loads are warp-collective,
                     // so every lane takes the same path
                     const bool win = __any_sync(0xffffffffu, jw > 0);
+                    const int ause = ring_uses(eg, kStages, U0) + myunit / kStages;
+                    if (!(ok = bwait(&sb->accfull[eg], ause & 1))) break;
+                    if (lq == 0) KVP_TSTAMP(n + i, 4);
+                    ptx::tc_fence_after();
+                    const int col0 = pp * p.n1;
+                    const int ncols = min(p.n1, p.rows - col0);
+                    const int nch = (ncols + 31) >> 5;
                     float acc = 0.f;
-                    bool mine = false;
-                    for (int pp = 0; pp < p.p1; ++pp, ++unit) {
-                        if ((unit & 1) != eg) continue;
-                        mine = true;
-                        const int st = unit & (kStages - 1);
-                        const int use = ring_uses(st, kStages, U0) + unit / kStages;
-                        if (!(ok = wait_phase(&sb->accfull[st], use & 1, sb, p, kErrWaitEpi))) break;
-                        if (lq == 0) KVP_TSTAMP(n + i, 4);
-                        ptx::tc_fence_after();
-                        const uint32_t tst = tlane + (uint32_t)(st * kStageCols);
-                        const int col0 = pp * p.n1;
-                        const int ncols = min(p.n1, p.rows - col0);
-                        const int nch = (ncols + 31) >> 5;
-                        auto proc = [&](const float (&v)[32], int c) {
-                            const int nrem = ncols - c * 32;
-                            acc += s1_chunk(v, lse2 + col0 + c * 32, wpos + col0 + c * 32,
-                                            win || nrem < 32, jw, nrem, p.scale2);
-                        };
-                        float x[32], y[32];
-                        __syncwarp();
-                        ptx::tmem_ld_32x32b_x32(tst, x);
-                        ptx::tmem_ld_wait(x);
 #pragma unroll 1
-                        for (int c = 0; c < nch; c += 2) {
-                            const bool h1 = c + 1 < nch, h2 = c + 2 < nch;
-                            if (h1) {
-                                __syncwarp();
-                                ptx::tmem_ld_32x32b_x32(tst + (c + 1) * 32, y);
-                            }
-                            proc(x, c);
-                            if (h1) {
-                                ptx::tmem_ld_wait(y);
-                                if (h2) {
-                                    __syncwarp();
-                                    ptx::tmem_ld_32x32b_x32(tst + (c + 2) * 32, x);
-                                }
-                                proc(y, c + 1);
-                                if (h2) ptx::tmem_ld_wait(x);
-                            }
-                        }
-                        ptx::tc_fence_before();
+                    for (int c = 0; c < nch; ++c) {
+                        float v[32];
                         __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&sb->accempty[st]);
-                        if (lq == 0) KVP_TSTAMP(n + i, 5);
+                        ptx::tmem_ld_32x32b_x32(tst + c * 32, v);
+                        ptx::tmem_ld_wait(v);
+                        const int nrem = ncols - c * 32;
+                        acc += s1_chunk(v, ls + col0 + c * 32, wpos + col0 + c * 32, win || nrem < 32,
+                                        jw, nrem, p.scale2);
                     }
-                    if (!ok || !mine) continue;
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&sb->accempty[eg]);
+                    if (lq == 0) KVP_TSTAMP(n + i, 5);
+                    const int cb = i & (kCombBufs - 1), cuse = i / kCombBufs;
                     if (p.p1 > 1) {
-                        // the tile's rows are split over both groups: the group of the last part
-                        // finishes the tile, the other hands over its partial S1
-                        const int fin = (i * p.p1 + p.p1 - 1) & 1;
-                        const int cb = i & (kCombBufs - 1), cuse = i / kCombBufs;
-                        if (eg != fin) {
-                            if (!(ok = wait_phase(&sb->combempty[cb], (cuse & 1) ^ 1, sb, p, kErrWaitEpi))) break;
-                            comb[cb * kTile + lq] = acc;
+                        // the tile's rows are split over p1 groups: the group of the last part
+                        // finishes the tile, the others hand over their partial S1
+                        if (pp != p.p1 - 1) {
+                            if (!(ok = bwait(&sb->combempty[cb], (cuse & 1) ^ 1))) break;
+                            comb[(cb * (kMaxParts - 1) + pp) * kTile + lq] = acc;
                             __syncwarp();
                             if (lane == 0) ptx::mbar_arrive(&sb->combfull[cb]);
                             continue;
                         }
-                        if (!(ok = wait_phase(&sb->combfull[cb], cuse & 1, sb, p, kErrWaitEpi))) break;
-                        acc += comb[cb * kTile + lq];
+                        // a plain wait: the part groups wait for their accumulators in waits
+                        // that take V pieces, so the V stream goes on meanwhile
+                        if (!(ok = wait_warp(&sb->combfull[cb], cuse & 1, sb, p, kErrWaitEpi))) break;
+                        float others = 0.f;
+                        for (int q = 0; q < p.p1 - 1; ++q) others += comb[(cb * (kMaxParts - 1) + q) * kTile + lq];
+                        acc += others;
                         __syncwarp();
                         if (lane == 0) ptx::mbar_arrive(&sb->combempty[cb]);
                     }
-                    const int e = i & (kS2Bufs - 1), suse = i / kS2Bufs;
-                    if (!(ok = wait_phase(&sb->s2full[e], suse & 1, sb, p, kErrWaitEpi))) break;
-                    const float s2v = s2buf[e * kTile + lq];
+                    // the tile's S2, once its V pieces are in the ring; then the ring row is
+                    // released (four warps of this group read it)
+                    const int rs = i & (kS2Ring - 1);
+                    if (!(ok = bwait(&sb->s2full[rs], (i / kS2Ring) & 1))) break;
+                    if (lq == 0) KVP_MSTAMP(i, 2);
+                    const float s2v = s2ring[rs * kTile + lq];
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&sb->s2empty[e]);
+                    if (lane == 0) ptx::mbar_arrive(&sb->s2empty[rs]);
                     if (j < p.L) {
                         const size_t o = (size_t)head * p.L + j;
                         p.score[o] = acc * s2v;
@@ -801,6 +877,11 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         if (p.s2) p.s2[o] = s2v;
                     }
                 }
+                if (!ok) break;
+                // this segment's lse2 is no longer read by this warp
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sb->lseempty[buf]);
+                ++k;
             }
         }
     }
@@ -881,17 +962,18 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.tiles_per_head = plan.tiles_per_head;
     p.total_tiles = plan.total_tiles;
     // the planned cut, or a flat cut over the SMs of a smaller device
-    p.cph = plan.grid <= sms ? plan.cph : 0;
-    p.grid = plan.grid <= sms ? plan.grid : sms;
-    // slots each head needs with this grid must fit the workspace's
-    {
-        const long long T = p.total_tiles;
+    if (plan.grid <= sms) {
+        p.grid = plan.grid;
+        p.cph = plan.cph;
+        p.nseg = plan.nseg;
+    } else {
+        p.grid = sms;
+        p.cph = 0;
+        p.nseg = 1;
+        // slots each head needs with this grid must fit the workspace's
         int need = 0;
-        for (int h = 0; h < s.batch * s.hkv; ++h) {
-            const long long f = (long long)h * p.tiles_per_head;
-            need = std::max(need, owner_of(f + p.tiles_per_head - 1, T, p.grid, p.tiles_per_head, p.cph) -
-                                      owner_of(f, T, p.grid, p.tiles_per_head, p.cph) + 1);
-        }
+        for (int h = 0; h < s.batch * s.hkv; ++h)
+            need = std::max(need, ctas_touching(h, p.total_tiles, p.grid, p.tiles_per_head, 0));
         if (need * kSlotsPerCta > plan.maxslots) return false;
     }
     p.maxslots = plan.maxslots;
@@ -901,22 +983,22 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.tile_bytes = (uint32_t)kTile * D * 2;
     p.extra_peers = g_extra_peers;
     p.wait_limit_ns = g_wait_limit_ns;
-    // shared memory: Q | ring slots | lse2 | comb | s2buf | stage0 | wpos | barriers
+    // shared memory: Q | ring slots | lse2 [2] | comb | S2 ring | phase 0 hand-off [2] | wpos | barriers
     // (+1 KB to align the base)
-    const size_t lse_bytes = (size_t)((plan.rows + 3) / 4 * 4) * sizeof(float);
-    const size_t comb_bytes = (size_t)kCombBufs * kTile * sizeof(float);
-    const size_t s2_bytes = (size_t)kS2Bufs * kTile * sizeof(float);
-    const size_t stage_bytes = (size_t)plan.rows * sizeof(float2);
+    const size_t lse_bytes = 2 * (size_t)((plan.rows + 3) / 4 * 4) * sizeof(float);
+    const size_t comb_bytes = (size_t)kCombBufs * (kMaxParts - 1) * kTile * sizeof(float);
+    const size_t stage_bytes = 2 * (size_t)kGroups * plan.rows * sizeof(float2);
+    const size_t s2_bytes = (size_t)kS2Ring * kTile * sizeof(float) + 16;
     const size_t wpos_bytes = (size_t)((plan.rows + 7) / 8 * 8) * sizeof(uint16_t);
     const size_t fixed = lse_bytes + comb_bytes + s2_bytes + stage_bytes + wpos_bytes + kBarBytes + 1024;
     if (p.q_bytes + fixed > (size_t)kSmemLimit) return false;
     p.ns = (int)std::min<size_t>(kMaxSlots, ((size_t)kSmemLimit - p.q_bytes - fixed) / p.tile_bytes);
     if (p.ns < 2) return false;
-    // phase 1: K comes again (mostly from L2), V from HBM gets the deeper share; a tile
-    // split into several parts holds its K slot longer, so one K slot can do
-    p.nk1 = (p.p1 > 1 && p.ns <= 3) ? 1 : 2;
-    p.nv1 = p.ns - p.nk1;
-    if (p.nv1 < 1) return false;
+    // phase 0 streams K through every slot; phase 1 gives V (from HBM) the deeper share and
+    // K (mostly from L2) two slots, or one when the ring is short
+    p.nk = p.ns >= 4 ? 2 : 1;
+    p.nv = p.ns - p.nk;
+    if (p.nv < 1) return false;
     p.off_slots = p.q_bytes;
     uint32_t off = p.off_slots + (uint32_t)p.ns * p.tile_bytes;
     p.off_lse = off;
@@ -1010,8 +1092,8 @@ void set_fault(int extra_peers, unsigned long long wait_limit_ns) {
 #ifdef KVP_TRACE
 int take_trace(unsigned long long* out) {
     if (cudaMemcpyFromSymbol(out, g_kvp_trace, sizeof(g_kvp_trace)) != cudaSuccess) return -1;
-    if (cudaMemcpyFromSymbol(out + 148 * 8, g_kvp_ttrace, sizeof(g_kvp_ttrace)) != cudaSuccess) return -1;
-    return cudaMemcpyFromSymbol(out + 148 * 8 + 4 * 64 * 8, g_kvp_mtrace, sizeof(g_kvp_mtrace)) == cudaSuccess ? 0 : -1;
+    if (cudaMemcpyFromSymbol(out + 148 * 12, g_kvp_ttrace, sizeof(g_kvp_ttrace)) != cudaSuccess) return -1;
+    return cudaMemcpyFromSymbol(out + 148 * 12 + 4 * 64 * 8, g_kvp_mtrace, sizeof(g_kvp_mtrace)) == cudaSuccess ? 0 : -1;
 }
 #endif
 

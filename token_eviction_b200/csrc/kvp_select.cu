@@ -5,6 +5,9 @@
 // [L - w, L) and the B - w highest scores among [0, L - w); equal scores go to the
 // lower position; the list is written in ascending position order.
 //
+// The policy variant (kvp_select_policy) keeps the first s positions (attention sinks) and
+// ranks the candidates [s, L - w) by a key formed from S1 and S2 (see SelSource).
+//
 // One thread-block cluster of kCl CTAs per row. Each CTA holds a contiguous slice of
 // the row's candidates in shared memory as order-preserving 32-bit keys (the fp32 bit
 // pattern with the sign handled so that unsigned order equals numeric order).
@@ -75,35 +78,81 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* ws) {
     return r;
 }
 
+// What a row is ranked by. Plain (s1 == nullptr): the score itself, over [0, L - w).
+// Policy: candidates [sinks, L - w), ranked by a key formed from S1 and S2 in fp32:
+//   pool(S1)[j] = max of S1 over [j - kernel/2, j + kernel/2] within [0, L - w)
+//   mode 0: pool(S1) * S2 (IEEE multiply, no flush of subnormal operands); 1: pool(S1);
+//   2: S2; a subnormal key counts as zero.
+// The first `sinks` positions are always kept.
+struct SelSource {
+    const float* score;
+    const float* s1;
+    const float* s2;
+    int sinks, kernel, mode;
+};
+
+__device__ __forceinline__ float mul_rn_noftz(float a, float b) {
+    float r;
+    asm("mul.rn.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// Order-preserving key of candidate j of a row (row pointers already offset).
+__device__ __forceinline__ uint32_t source_key(const SelSource& src, const float* srow, const float* s1row,
+                                               const float* s2row, int j, int n) {
+    if (srow) return order_key(__float_as_uint(__ldg(srow + j)));
+    float key;
+    if (src.mode == 2) {
+        key = __ldg(s2row + j);
+    } else {
+        // S1 >= 0: the largest bit pattern is the largest value, subnormals included
+        const int half = src.kernel >> 1;
+        uint32_t pooled = __float_as_uint(__ldg(s1row + j));
+        for (int t = max(0, j - half); t <= min(n - 1, j + half); ++t)
+            pooled = max(pooled, __float_as_uint(__ldg(s1row + t)));
+        key = src.mode == 1 ? __uint_as_float(pooled) : mul_rn_noftz(__uint_as_float(pooled), __ldg(s2row + j));
+    }
+    uint32_t bits = __float_as_uint(key);
+    if ((bits & 0x7F800000u) == 0u) bits = 0u;     // zero or subnormal: zero
+    return order_key(bits);
+}
+
 template <bool kInSmem>
 __global__ void __launch_bounds__(kSelThreads, 1)
-select_cluster(const float* __restrict__ score, int32_t* __restrict__ idx, int L, int w, int B,
-               int slice) {
+select_cluster(const SelSource src, int32_t* __restrict__ idx, int L, int w, int B, int slice) {
     extern __shared__ uint32_t keys[];   // [slice] when kInSmem
     __shared__ SelShared sh;
     cg::cluster_group cluster = cg::this_cluster();
     const unsigned rank = cluster.block_rank();
     const int row = blockIdx.x / kCl;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = L - w, kk = B - w;
-    const uint32_t* rowbits = reinterpret_cast<const uint32_t*>(score + (size_t)row * L);
+    const int n = L - w, s0 = src.sinks, kk = B - w - s0;
+    // plain when score is given; otherwise a policy key (s1 is NULL when mode 2 ranks by S2)
+    const float* srow = src.score ? src.score + (size_t)row * L : nullptr;
+    const float* s1row = src.s1 ? src.s1 + (size_t)row * L : nullptr;
+    const float* s2row = src.s2 ? src.s2 + (size_t)row * L : nullptr;
     int32_t* out = idx + (size_t)row * B;
 
-    if (rank == 0)
-        for (int t = tid; t < w; t += kSelThreads) out[kk + t] = n + t;
+    // sinks, then the kk selected candidates, then the window: all ascending
+    if (rank == 0) {
+        for (int t = tid; t < s0; t += kSelThreads) out[t] = t;
+        for (int t = tid; t < w; t += kSelThreads) out[s0 + kk + t] = n + t;
+    }
+    out += s0;
     if (kk == 0) return;                  // same decision in every CTA of the cluster
-    if (kk == n) {
-        for (int t = (int)rank * kSelThreads + tid; t < n; t += kCl * kSelThreads) out[t] = t;
+    if (kk == n - s0) {
+        for (int t = (int)rank * kSelThreads + tid; t < n - s0; t += kCl * kSelThreads) out[t] = s0 + t;
         return;
     }
 
-    const int lo = min(n, (int)rank * slice), hi = min(n, lo + slice);
+    // this CTA's slice of the candidates [s0, n)
+    const int lo = min(n, s0 + (int)rank * slice), hi = min(n, lo + slice);
     auto key_at = [&](int j) -> uint32_t {  // j in [lo, hi)
         if (kInSmem) return keys[j - lo];
-        return order_key(__ldg(rowbits + j));
+        return source_key(src, srow, s1row, s2row, j, n);
     };
     if (kInSmem) {
-        for (int j = lo + tid; j < hi; j += kSelThreads) keys[j - lo] = order_key(__ldg(rowbits + j));
+        for (int j = lo + tid; j < hi; j += kSelThreads) keys[j - lo] = source_key(src, srow, s1row, s2row, j, n);
     }
     SelShared* leader = cluster.map_shared_rank(&sh, 0);
 
@@ -235,12 +284,11 @@ select_cluster(const float* __restrict__ score, int32_t* __restrict__ idx, int L
 
 }  // namespace
 
-cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score, int32_t* idx,
-                          void* scratch, cudaStream_t st) {
-    (void)p;
-    (void)scratch;
-    const int n = s.seq_len - s.window;
-    const int slice = (n + kCl - 1) / kCl;
+namespace {
+
+cudaError_t launch_select_source(const kvp_shape& s, const SelSource& src, int32_t* idx, cudaStream_t st) {
+    const int nc = s.seq_len - s.window - src.sinks;      // candidates
+    const int slice = (nc + kCl - 1) / kCl;
     const bool in_smem = slice <= kSliceCap;
     const size_t dyn = in_smem ? (size_t)slice * sizeof(uint32_t) : 0;
     cudaLaunchConfig_t cfg = {};
@@ -258,11 +306,25 @@ cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score,
     cudaError_t e;
     if (in_smem) {
         if ((e = allow_dynamic_smem((const void*)select_cluster<true>, dyn)) != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, select_cluster<true>, score, idx, s.seq_len, s.window,
-                                  s.budget, slice);
+        return cudaLaunchKernelEx(&cfg, select_cluster<true>, src, idx, s.seq_len, s.window, s.budget, slice);
     }
-    return cudaLaunchKernelEx(&cfg, select_cluster<false>, score, idx, s.seq_len, s.window,
-                              s.budget, slice);
+    return cudaLaunchKernelEx(&cfg, select_cluster<false>, src, idx, s.seq_len, s.window, s.budget, slice);
+}
+
+}  // namespace
+
+cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score, int32_t* idx,
+                          void* scratch, cudaStream_t st) {
+    (void)p;
+    (void)scratch;
+    const SelSource src = {score, nullptr, nullptr, 0, 1, 0};
+    return launch_select_source(s, src, idx, st);
+}
+
+cudaError_t launch_select_policy(const kvp_shape& s, const kvp_policy& pol, const float* s1,
+                                 const float* s2, int32_t* idx, cudaStream_t st) {
+    const SelSource src = {nullptr, s1, s2, pol.sinks, pol.pool_kernel, pol.mode};
+    return launch_select_source(s, src, idx, st);
 }
 
 #ifdef KVP_CHECKS
