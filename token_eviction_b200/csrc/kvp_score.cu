@@ -210,18 +210,6 @@ __device__ __forceinline__ float row_absmax(const uint8_t* row, int lane) {
 __device__ __forceinline__ int ring_uses(int s, int period, int n) {
     return n > s ? (n - s + period - 1) / period : 0;
 }
-// K slot of the run's tile i in `phase`, and the number of that slot's earlier K loads.
-// Phase 0 streams K through all ns slots in turn; phase 1 through slots [0, nk).
-__device__ __forceinline__ int k_slot(int phase, int i, int n, const Params& p, int& use) {
-    if (phase == 0) {
-        use = i / p.ns;
-        return i % p.ns;
-    }
-    const int s = i % p.nk;
-    use = ring_uses(s, p.ns, n) + i / p.nk;
-    return s;
-}
-
 // The CTA's work in one phase: its segments in order, each split where it crosses a KV
 // head (only flat runs do), with the slot of the CTA's partial in that head.
 // Tile numbers fit in 32 bits (the plan checks it).
@@ -372,7 +360,7 @@ __device__ __forceinline__ void v_worker(uint8_t* smem, const Params& p, int n, 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-               const __grid_constant__ CUtensorMap vmap, const Params p) {
+               const __grid_constant__ CUtensorMap vmap, const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* Qs = smem;                                  // [D / 64][qrows][64] bf16, 128B swizzle
@@ -393,10 +381,17 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int n = 0;                                      // tiles in this CTA's run
-    for (int s = 0; s < p.nseg; ++s) {
-        uint32_t b, e;
-        segment_of_u32(blockIdx.x, s, p.total_tiles, p.grid, p.tiles_per_head, p.cph, b, e);
-        n += (int)(e - b);
+    int seg_head0 = -1, seg_head1 = -1;             // KV head of each segment's first tile
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        if (s < p.nseg) {
+            uint32_t b, e;
+            segment_of_u32(blockIdx.x, s, p.total_tiles, p.grid, p.tiles_per_head, p.cph, b, e);
+            n += (int)(e - b);
+            const int h = e > b ? (int)(b / (uint32_t)p.tiles_per_head) : -1;
+            if (s == 0) seg_head0 = h;
+            else seg_head1 = h;
+        }
     }
     const int U0 = n * p.u0;                        // phase 0 units of the run
 
@@ -470,9 +465,15 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const uint64_t pol_keep = ptx::policy_evict_normal();
         const uint64_t pol_stream = ptx::policy_evict_first();
         int qgen = 0, cur = -1;
-        int kiss[kMaxSlots] = {}, viss[kMaxSlots] = {};     // loads issued per slot
+        // per slot, in registers: bit s = parity of the loads issued to it, and whether any was
+        uint32_t kpar = 0, kused = 0, vpar = 0, vused = 0;
+        int vs = 0;                                         // next V slot (index s - nk)
         bool ok = true;
         for (int phase = 0; phase < 2 && ok; ++phase) {
+            // K goes round slots [0, ns) in phase 0 and [0, nk) in phase 1; the parity of a
+            // slot's loads so far gives the phase of its barriers
+            const int kring = phase == 0 ? p.ns : p.nk;
+            int ks = 0;
             CtaRun it(p);
             int head, slot, a, b;
             int i = 0;                                      // tile number within the run
@@ -490,26 +491,30 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 }
                 for (int t = a; t < b; ++t, ++i) {
                     const int key0 = (t - head * p.tiles_per_head) * kTile;
-                    int use;
-                    const int s = k_slot(phase, i, n, p, use);
-                    if (!(ok = wait_phase(&sb->kempty[s], (use & 1) ^ 1, sb, p, kErrWaitTma))) break;
+                    const int s = ks;
+                    ks = ks + 1 == kring ? 0 : ks + 1;
+                    if (!(ok = wait_phase(&sb->kempty[s], ((kpar >> s) & 1) ^ 1, sb, p, kErrWaitTma))) break;
                     KVP_TSTAMP(phase * n + i, 0);
                     ptx::mbar_arrive_expect_tx(&sb->kfull[s], p.tile_bytes);
                     for (int c = 0; c < kHalves; ++c)
                         ptx::tma_load_3d(Slots + s * kSlotBytes + c * kHalfTile, &kmap, &sb->kfull[s],
                                          c * 64, key0, head, phase == 0 ? pol_keep : pol_stream);
-                    ++kiss[s];
+                    kpar ^= 1u << s;
+                    kused |= 1u << s;
                     if (phase == 1) {
-                        const int jv = i % p.nv, sv = p.nk + jv, vuse = i / p.nv;
+                        const int jv = vs, sv = p.nk + jv;
+                        vs = vs + 1 == p.nv ? 0 : vs + 1;
                         // a V slot's first load waits for its last K load of phase 0 to be consumed
-                        const int u0s = vuse == 0 ? ring_uses(sv, p.ns, n) : 0;
-                        if (u0s > 0 && !(ok = wait_phase(&sb->kempty[sv], (u0s - 1) & 1, sb, p, kErrWaitTma))) break;
-                        if (!(ok = wait_phase(&sb->vempty[jv], (vuse & 1) ^ 1, sb, p, kErrWaitTma))) break;
+                        if (!((vused >> jv) & 1) && ((kused >> sv) & 1) &&
+                            !(ok = wait_phase(&sb->kempty[sv], ((kpar >> sv) & 1) ^ 1, sb, p, kErrWaitTma)))
+                            break;
+                        if (!(ok = wait_phase(&sb->vempty[jv], ((vpar >> jv) & 1) ^ 1, sb, p, kErrWaitTma))) break;
                         KVP_TSTAMP(n + i, 6);
                         ptx::mbar_arrive_expect_tx(&sb->vfull[jv], p.tile_bytes);
                         ptx::tma_load_3d(Slots + sv * kSlotBytes, &vmap, &sb->vfull[jv], 0, key0, head,
                                          pol_stream);
-                        ++viss[jv];
+                        vpar ^= 1u << jv;
+                        vused |= 1u << jv;
                     }
                 }
             }
@@ -518,9 +523,9 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         // Never leave with copies in flight: wait for the last load issued to every slot
         // (these waits do not stop early when the CTA unwinds).
         for (int s = 0; s < p.ns; ++s)
-            if (kiss[s] > 0) drain_wait(&sb->kfull[s], (kiss[s] - 1) & 1);
+            if ((kused >> s) & 1) drain_wait(&sb->kfull[s], ((kpar >> s) & 1) ^ 1);
         for (int jv = 0; jv < p.nv; ++jv)
-            if (viss[jv] > 0) drain_wait(&sb->vfull[jv], (viss[jv] - 1) & 1);
+            if ((vused >> jv) & 1) drain_wait(&sb->vfull[jv], ((vpar >> jv) & 1) ^ 1);
         if (qgen > 0) drain_wait(&sb->qfull, (qgen - 1) & 1);
       }
     } else if (warp == 1) {
@@ -529,8 +534,12 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             const uint32_t q_addr = ptx::smem_u32(Qs), k_addr = ptx::smem_u32(Slots);
             const uint32_t idesc0 = ptx::idesc_bf16_f32(128, p.nk0);
             int qgen = 0, cur = -1;
+            uint32_t kpar = 0;                              // bit s: parity of slot s's loads consumed
+            uint32_t apar = 0;                              // bit st: parity of stage st's units
             bool ok = true;
             for (int phase = 0; phase < 2 && ok; ++phase) {
+                const int kring = phase == 0 ? p.ns : p.nk;   // the producer's slot order
+                int ks = 0;
                 CtaRun it(p);
                 int head, slot, a, b;
                 int i = 0;                                  // tile number within the run
@@ -543,21 +552,22 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         ptx::tc_fence_after();
                     }
                     for (int t = a; t < b && ok; ++t, ++i) {
-                        int kuse;
-                        const int s = k_slot(phase, i, n, p, kuse);
-                        if (!(ok = wait_phase(&sb->kfull[s], kuse & 1, sb, p, kErrWaitMma))) break;
+                        const int s = ks;
+                        ks = ks + 1 == kring ? 0 : ks + 1;
+                        if (!(ok = wait_phase(&sb->kfull[s], (kpar >> s) & 1, sb, p, kErrWaitMma))) break;
                         KVP_TSTAMP(phase * n + i, 1);
                         const uint32_t kbase = k_addr + s * kSlotBytes;
                         const int nunits = phase == 0 ? p.u0 : p.p1;
                         for (int j = 0; j < nunits; ++j, ++unit) {
                             const int st = unit & (kStages - 1);
-                            const int use = (phase == 0 ? 0 : ring_uses(st, kStages, U0)) + unit / kStages;
-                            if (!(ok = wait_phase(&sb->accempty[st], (use & 1) ^ 1, sb, p, kErrWaitMma))) break;
+                            if (!(ok = wait_phase(&sb->accempty[st], ((apar >> st) & 1) ^ 1, sb, p, kErrWaitMma))) break;
+                            apar ^= 1u << st;
                             if (j == 0) KVP_TSTAMP(phase * n + i, 2);
                             ptx::tc_fence_after();
                             const uint32_t d0 = tmem + (uint32_t)(st * kStageCols);
                             if (phase == 0) {
                                 // D[row, key] for every row block: A = Q rows, B = the unit's keys
+#pragma unroll 1
                                 for (int rb = 0; rb < p.nrb; ++rb) {
                                     const uint64_t qd = ptx::sw128_kmajor_desc(q_addr + rb * 128 * 128);
                                     const uint64_t kd = ptx::sw128_kmajor_desc(kbase + j * p.nk0 * 128);
@@ -585,19 +595,18 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         }
                         if (!ok) break;
                         ptx::mma_commit(&sb->kempty[s]);
+                        kpar ^= 1u << s;
                         KVP_TSTAMP(phase * n + i, 3);
                     }
                     if (!ok) break;
-                    // release the query rows when the next segment loads another head's
+                    // release the query rows when the next piece of work (this segment's next
+                    // head, the next segment, or phase 1's first) is another head's
                     {
-                        CtaRun peek = it;
-                        int nh = -1, ns2, na, nb;
-                        bool more = peek.next(nh, na, nb, ns2);
-                        if (!more && phase == 0) {
-                            CtaRun again(p);
-                            more = again.next(nh, na, nb, ns2);
-                        }
-                        if (more && nh != cur) ptx::mma_commit(&sb->qempty);
+                        int nh;
+                        if (it.t < it.end) nh = it.t / p.tiles_per_head;
+                        else if (it.s + 1 < p.nseg) nh = seg_head1;     // nseg <= 2
+                        else nh = phase == 0 ? seg_head0 : -1;
+                        if (nh >= 0 && nh != cur) ptx::mma_commit(&sb->qempty);
                     }
                 }
                 KVP_STAMP(3 + phase);
@@ -607,12 +616,13 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             ptx::mma_commit(&sb->fin);
             drain_wait(&sb->fin, 0);
         }
-    } else if (warp == kWarpPub) {
+    } else if (warp == kWarpPub || warp == kWarpV) {
+      bool ok = true;
+      if (warp == kWarpPub) {
         // ------------------------------------------------------------ phase 0 publisher
         // Per segment: combine the epilogue groups' (m, l) of every row, write the CTA's
         // slot, then bump the head's completion counter (so that no epilogue thread waits on
         // a global fence).
-        bool ok = true;
         CtaRun it(p);
         int head, slot, a, b;
         int k = 0;
@@ -645,10 +655,9 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             ++k;
         }
         if (lane == 0) KVP_STAMP(5);
-        if (ok) v_worker<D>(smem, p, n, sb);
-    } else if (warp == kWarpV) {
-        // ------------------------------------------------------------ V pieces
-        v_worker<D>(smem, p, n, sb);
+      }
+      // ------------------------------------------------------------ V pieces (warps 2 and 3)
+      if (ok) v_worker<D>(smem, p, n, sb);
     } else if (warp >= kWarpEpi) {
         // ------------------------------------------------------------ epilogue (warps 4-19)
         const int et = threadIdx.x - 32 * kWarpEpi;      // 0 .. kEpiThreads-1
