@@ -135,6 +135,25 @@ KVP_API kvp_status kvp_select_policy(const kvp_shape* shape, const kvp_policy* p
                                      const float* s1, const float* s2, int32_t* idx, void* stream);
 
 /*
+ * CurDKV leverage scores (CurDKV rebuttal page, "A clearer description of Algorithm 1",
+ * steps 1-4), an alternative to kvp_score for the same selection and compaction:
+ *   lk_j = ||K_j G||^2, lv_j = ||V_j G||^2   (squared row norms of the projected key and
+ *                                             value of position j)
+ *   score_j = lk_j * lv_j / sum over the KV head's L positions of lk * lv   (0 if that is 0)
+ *   k, v   [b, hkv, L, d] bf16
+ *   g      [d, r] bf16: the Gaussian projection, drawn by the caller; 1 <= r <= 32
+ *   score  [b, hkv, L] fp32 output (sums to 1 per (b, KV head))
+ *   workspace  as for kvp_score (kvp_workspace_bytes); its error word is cleared and set
+ *              as by kvp_score (kvp_workspace_status reads it)
+ * Arithmetic: bf16 products accumulated in fp32 on the tensor cores, fp32 squares, sums
+ * and product; the normalising sum is taken in a fixed order (repeat calls agree bit for
+ * bit). Rank with kvp_select_policy in KVP_RANK_S1 mode (score as s1), with CurDKV's sinks.
+ */
+KVP_API kvp_status kvp_leverage(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
+                                const uint16_t* g, int32_t r, float* score, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
  * Compaction: k_out[b, h, t, :] = k[b, h, idx[b, h, t], :], the same for v; a bit copy.
  *   k, v          [b, hkv, L, d] bf16
  *   idx           [b, hkv, B]    int32, entries in [0, L) (an entry outside that range

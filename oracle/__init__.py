@@ -52,6 +52,8 @@ def _get():
         lib.oracle_compact.restype = i
         lib.oracle_select_policy.argtypes = [i, i, i, i, i, i, i, i, p, p, p, p]
         lib.oracle_select_policy.restype = i
+        lib.oracle_leverage.argtypes = [i, i, i, i, p, p, p, p, p, p]
+        lib.oracle_leverage.restype = i
         _lib = lib
     return _lib
 
@@ -141,3 +143,24 @@ def oracle_layer(q_win, k, v, window: int, budget: int):
     idx = oracle_select(s, window, budget)
     k_out, v_out = oracle_compact(k, v, idx)
     return {"s1": s1, "s2": s2, "score": s, "idx": idx, "k_out": k_out, "v_out": v_out}
+
+
+def oracle_leverage(k, v, g, want_parts: bool = False):
+    """CurDKV leverage scores [..., L] (float64): squared row norms of K G and V G, their
+    product, normalised to sum 1 over each row's positions (CurDKV rebuttal page,
+    "A clearer description of Algorithm 1", steps 1-4). k, v [..., L, d] and g [d, r]:
+    bf16 bit patterns. With ``want_parts`` also returns the two squared norms."""
+    k, v, g = _u16(k), _u16(v), _u16(g)
+    assert k.shape == v.shape and g.ndim == 2 and g.shape[0] == k.shape[-1]
+    lead, L, d = k.shape[:-2], k.shape[-2], k.shape[-1]
+    r = g.shape[1]
+    rows = int(np.prod(lead)) if lead else 1
+    score = np.empty(lead + (L,))
+    lk = np.empty(lead + (L,)) if want_parts else None
+    lv = np.empty(lead + (L,)) if want_parts else None
+    rc = _get().oracle_leverage(rows, L, d, r, k.ctypes.data, v.ctypes.data, g.ctypes.data,
+                                None if lk is None else lk.ctypes.data,
+                                None if lv is None else lv.ctypes.data, score.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_leverage: bad size")
+    return (score, lk, lv) if want_parts else score

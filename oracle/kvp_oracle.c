@@ -36,10 +36,20 @@
  * review; read here as SnapKV's 1-D max pooling of S1 over the positions before the window,
  * the kernel centred on each position, positions past either end left out).
  *
+ * CurDKV leverage scores (oracle_leverage), the CurDKV rebuttal page, "A clearer
+ * description of Algorithm 1", steps 1-4, for one KV head's K and V (L x d each):
+ *   project both rows with the caller's Gaussian G (d x r); a row's leverage score is its
+ *   row norm after the projection; the key and value scores are combined and normalised.
+ * Readings: the row norm is the squared Euclidean norm (leverage scores are squared row
+ * norms); "combined" is the product lk_j * lv_j (as SlimKV combines S1 and S2); the
+ * normalisation divides by the sum over the head's L positions (all zero if that is 0).
+ *
  * Parity pins (tests): sum_j S1 = G w; closed forms for identical keys and for a
  * single planted key; G = 1, w = 1 against a library softmax; brute force on tiny
  * inputs; selection against a library stable sort; gather against library indexing;
- * pooling against a library sliding maximum and a planted spike.
+ * pooling against a library sliding maximum and a planted spike; leverage scores against
+ * library row norms for an identity projection, a rank-one closed form, brute force on
+ * tiny inputs and their invariants (sum 1, scale and permutation).
  */
 #include <math.h>
 #include <stdint.h>
@@ -242,5 +252,45 @@ int oracle_select_policy(int rows, int L, int w, int B, int sinks, int kernel, i
         free(c);
         free(key);
     }
+    return 0;
+}
+
+/*
+ * CurDKV leverage scores of every position of `rows` (sequence, KV head) rows.
+ *   k, v   [rows][L][d] bf16 bits;  g [d][r] bf16 bits
+ *   lk, lv [rows][L] squared norms of K_j G and V_j G (may be NULL)
+ *   score  [rows][L] lk * lv / sum over the row's positions of lk * lv
+ * Returns 0, or -1 on a bad size.
+ */
+int oracle_leverage(int rows, int L, int d, int r, const uint16_t* k, const uint16_t* v,
+                    const uint16_t* g, double* lk, double* lv, double* score) {
+    if (rows < 0 || L < 1 || d < 1 || r < 1) return -1;
+    double* gd = (double*)malloc(sizeof(double) * (size_t)d * r);
+    for (size_t t = 0; t < (size_t)d * r; ++t) gd[t] = widen_bf16(g[t]);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int row = 0; row < rows; ++row) {
+        const uint16_t* K = k + (size_t)row * L * d;
+        const uint16_t* V = v + (size_t)row * L * d;
+        double* out = score + (size_t)row * L;
+        double total = 0.0;
+        for (int j = 0; j < L; ++j) {
+            double nk = 0.0, nv = 0.0;
+            for (int c = 0; c < r; ++c) {
+                double pk = 0.0, pv = 0.0;               /* (K_j G)_c and (V_j G)_c */
+                for (int t = 0; t < d; ++t) {
+                    pk += widen_bf16(K[(size_t)j * d + t]) * gd[(size_t)t * r + c];
+                    pv += widen_bf16(V[(size_t)j * d + t]) * gd[(size_t)t * r + c];
+                }
+                nk += pk * pk;
+                nv += pv * pv;
+            }
+            if (lk) lk[(size_t)row * L + j] = nk;
+            if (lv) lv[(size_t)row * L + j] = nv;
+            out[j] = nk * nv;
+            total += out[j];
+        }
+        for (int j = 0; j < L; ++j) out[j] = total > 0.0 ? out[j] / total : 0.0;
+    }
+    free(gd);
     return 0;
 }

@@ -361,3 +361,71 @@ def test_bad_policies_raise():
     for kw in (dict(sinks=45), dict(sinks=-1), dict(kernel=4), dict(kernel=0), dict(mode=3)):
         with pytest.raises(ValueError):
             oracle.oracle_select_policy(s, s, 8, 40, **kw)
+
+
+# ---- CurDKV leverage scores (CurDKV rebuttal page, "A clearer description of Algorithm 1")
+
+def lev_inputs(rows, L, d, r, seed):
+    k = synth.normal_bf16(rows * L, d, seed, 1).reshape(rows, L, d)
+    v = synth.normal_bf16(rows * L, d, seed, 2).reshape(rows, L, d)
+    g = synth.normal_bf16(d, r, seed, 3)
+    return k, v, g
+
+
+def test_leverage_identity_projection_gives_library_row_norms():
+    """G = I (r = d): the projected rows are the rows themselves, so the key and value
+    scores are numpy's squared row norms, and the combined score their normalised product."""
+    d, L = 16, 50
+    k, v, _ = lev_inputs(2, L, d, d, seed=11)
+    g = bf16(np.eye(d))
+    score, lk, lv = oracle.oracle_leverage(k, v, g, want_parts=True)
+    nk = np.linalg.norm(f64(k), axis=-1) ** 2
+    nv = np.linalg.norm(f64(v), axis=-1) ** 2
+    np.testing.assert_allclose(lk, nk, rtol=1e-13)
+    np.testing.assert_allclose(lv, nv, rtol=1e-13)
+    prod = nk * nv
+    np.testing.assert_allclose(score, prod / prod.sum(-1, keepdims=True), rtol=1e-12)
+
+
+def test_leverage_rank_one_projection_closed_form():
+    """r = 1 with G = g: the key score is (K_j . g)^2, a dot product numpy computes; a
+    transposed G, a dropped square or a sum in place of the product fails this."""
+    d, L = 32, 40
+    k, v, _ = lev_inputs(1, L, d, 1, seed=12)
+    gcol = bf16(np.linspace(-1.5, 2.0, d))
+    score, lk, lv = oracle.oracle_leverage(k, v, gcol.reshape(d, 1), want_parts=True)
+    gv = f64(gcol)
+    ek = (f64(k[0]) @ gv) ** 2
+    ev = (f64(v[0]) @ gv) ** 2
+    np.testing.assert_allclose(lk[0], ek, rtol=1e-12)
+    np.testing.assert_allclose(lv[0], ev, rtol=1e-12)
+    np.testing.assert_allclose(score[0], ek * ev / np.sum(ek * ev), rtol=1e-12)
+
+
+def test_leverage_brute_force_tiny():
+    d, L, r = 5, 7, 3
+    k, v, g = lev_inputs(1, L, d, r, seed=13)
+    K, V, G = f64(k[0]), f64(v[0]), f64(g)
+    comb = []
+    for j in range(L):
+        nk = math.fsum(math.fsum(K[j, t] * G[t, c] for t in range(d)) ** 2 for c in range(r))
+        nv = math.fsum(math.fsum(V[j, t] * G[t, c] for t in range(d)) ** 2 for c in range(r))
+        comb.append(nk * nv)
+    total = math.fsum(comb)
+    np.testing.assert_allclose(oracle.oracle_leverage(k, v, g)[0], [c / total for c in comb], rtol=1e-12)
+
+
+def test_leverage_invariants():
+    """Scores sum to 1 per row; scaling G by 2 (exact in bf16) leaves them unchanged;
+    permuting the positions permutes them; a zero key row scores 0."""
+    d, L, r = 64, 300, 20
+    k, v, g = lev_inputs(3, L, d, r, seed=14)
+    s = oracle.oracle_leverage(k, v, g)
+    np.testing.assert_allclose(s.sum(-1), 1.0, rtol=1e-12)
+    g2 = bf16(2.0 * f64(g))
+    np.testing.assert_allclose(oracle.oracle_leverage(k, v, g2), s, rtol=1e-12)
+    perm = np.random.default_rng(3).permutation(L)
+    np.testing.assert_allclose(oracle.oracle_leverage(k[:, perm], v[:, perm], g), s[:, perm], rtol=1e-12)
+    kz = k.copy()
+    kz[1, 17] = 0
+    assert oracle.oracle_leverage(kz, v, g)[1, 17] == 0.0

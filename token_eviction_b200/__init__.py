@@ -11,6 +11,7 @@ The functions carry the C names:
 * ``kvp_score(shape, q_win, k, v, score, s1=None, s2=None, workspace=None, stream=None)``
 * ``kvp_select(shape, score, idx, workspace=None, stream=None)``
 * ``kvp_select_policy(shape, policy, s1, s2, idx, stream=None)``
+* ``kvp_leverage(shape, k, v, g, score, workspace=None, stream=None)``
 * ``kvp_compact(shape, k, v, idx, k_out, v_out, stream=None)``
 * ``kvp_workspace_status(workspace, stream=None)``
 * ``kvp_status_string(status)``
@@ -84,6 +85,8 @@ def _load():
     lib.kvp_select.restype = ctypes.c_int
     lib.kvp_select_policy.argtypes = [S, ctypes.POINTER(KvpPolicy), P, P, P, P]
     lib.kvp_select_policy.restype = ctypes.c_int
+    lib.kvp_leverage.argtypes = [S, P, P, P, ctypes.c_int32, P, P, ctypes.c_size_t, P]
+    lib.kvp_leverage.restype = ctypes.c_int
     lib.kvp_compact.argtypes = [S, P, P, P, P, P, P]
     lib.kvp_compact.restype = ctypes.c_int
     lib.kvp_status_string.argtypes = [ctypes.c_int]
@@ -106,7 +109,8 @@ _lib = _load()
 # enqueues one small memset of its workspace counters.
 KERNELS_PER_LAYER = 3
 
-EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_select_policy", "kvp_compact",
+EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_select_policy", "kvp_leverage",
+            "kvp_compact",
             "kvp_workspace_status",
             "kvp_score_static", "kvp_score_static_status", "kvp_status_string", "kvp_last_cuda_error")
 
@@ -217,6 +221,25 @@ def kvp_select_policy(shape, policy, s1, s2, idx, stream=None):
     st = _lib.kvp_select_policy(ctypes.byref(sh), ctypes.byref(pol), p1, p2, pi, _stream(stream))
     if st != KVP_OK:
         raise KvpError(st, "kvp_select_policy")
+
+
+def kvp_leverage(shape, k, v, g, score, workspace=None, stream=None):
+    """CurDKV leverage scores of every position: squared row norms of K G and V G, their
+    product, normalised per KV head. g: [d, r] bf16 CUDA tensor, 1 <= r <= 32."""
+    sh = _as_shape(shape)
+    b, hkv, d, L = sh.batch, sh.hkv, sh.head_dim, sh.seq_len
+    if not isinstance(g, torch.Tensor) or g.dim() != 2 or g.shape[0] != d:
+        raise ValueError(f"g must be a [{d}, r] tensor")
+    args = (_ptr(k, "k", torch.bfloat16, (b, hkv, L, d)),
+            _ptr(v, "v", torch.bfloat16, (b, hkv, L, d)),
+            _ptr(g, "g", torch.bfloat16, tuple(g.shape)))
+    ps = _ptr(score, "score", torch.float32, (b, hkv, L))
+    if workspace is None:
+        workspace = workspace_for(sh, k.device)
+    st = _lib.kvp_leverage(ctypes.byref(sh), *args, int(g.shape[1]), ps, workspace.data_ptr(),
+                           workspace.numel(), _stream(stream))
+    if st != KVP_OK:
+        raise KvpError(st, "kvp_leverage")
 
 
 def kvp_compact(shape, k, v, idx, k_out, v_out, stream=None):

@@ -132,6 +132,24 @@ extern "C" kvp_status kvp_select_policy(const kvp_shape* shape, const kvp_policy
     return KVP_OK;
 }
 
+extern "C" kvp_status kvp_leverage(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
+                                   const uint16_t* g, int32_t r, float* score, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    if (!shape || !k || !v || !g || !score) return KVP_ERR_NULL;
+    Plan p;
+    if (!plan_of(*shape, &p)) return KVP_ERR_SHAPE;
+    if (r < 1 || r > 32) return KVP_ERR_SHAPE;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(score) || ((uintptr_t)g & 1u)) return KVP_ERR_ALIGN;
+    if (!workspace || workspace_bytes < p.bytes) return KVP_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KVP_ERR_ALIGN;
+    int maxparts = 0;
+    const int grid = std::min(kPlanGrid, p.total_tiles);
+    if (p.off_part + leverage_part_bytes(*shape, p, grid, &maxparts) > p.off_select) return KVP_ERR_SHAPE;
+    const cudaError_t e = launch_leverage(*shape, p, k, v, g, r, score, workspace, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_failed(e);
+    return KVP_OK;
+}
+
 extern "C" kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
                                   const int32_t* idx, uint16_t* k_out, uint16_t* v_out,
                                   void* stream) {
@@ -161,13 +179,15 @@ extern "C" KVP_API void kvp_debug_set_fault(int extra_peers, unsigned long long 
 
 // Debug builds only: copy out (and clear) the first failed device-side bounds check.
 extern "C" KVP_API int kvp_debug_take_check_unit(int unit, int* out4) {
-    int (*readers[3])(int*) = {take_check_score, take_check_select, take_check_compact};
-    if (unit < 0 || unit > 2) return -1;
+    int (*readers[4])(int*) = {take_check_score, take_check_select, take_check_compact,
+                               take_check_leverage};
+    if (unit < 0 || unit > 3) return -1;
     return readers[unit](out4);
 }
 
 extern "C" KVP_API int kvp_debug_take_check(int* out4) {
-    int (*readers[3])(int*) = {take_check_score, take_check_select, take_check_compact};
+    int (*readers[4])(int*) = {take_check_score, take_check_select, take_check_compact,
+                               take_check_leverage};
     out4[0] = out4[1] = out4[2] = out4[3] = 0;
     for (auto rd : readers) {
         int v[4];

@@ -1,6 +1,7 @@
 // Internal declarations shared by the kvp CUDA translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -124,10 +125,20 @@ cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score,
                           void* scratch, cudaStream_t st);
 cudaError_t launch_select_policy(const kvp_shape& s, const kvp_policy& pol, const float* s1,
                                  const float* s2, int32_t* idx, cudaStream_t st);
+cudaError_t launch_leverage(const kvp_shape& s, const Plan& p, const uint16_t* k, const uint16_t* v,
+                            const uint16_t* g, int r, float* score, void* workspace, cudaStream_t st);
+// Bytes of the leverage kernel's partial sums with `grid` CTAs (they live in the
+// workspace's partial-softmax region) and the slots per KV head.
+size_t leverage_part_bytes(const kvp_shape& s, const Plan& p, int grid, int* maxparts);
 cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t* v,
                            const int32_t* idx, uint16_t* k_out, uint16_t* v_out, cudaStream_t st);
 
 int num_sms();
+
+// A bf16 tensor map of `rank` dimensions (innermost first) with tile box `box`; false if
+// the driver's encoder is unavailable or rejects the layout.
+bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle swz);
 
 // Records `e` as the calling thread's last CUDA error (what kvp_last_cuda_error() names),
 // clears the runtime's sticky copy of a launch error, and returns KVP_ERR_CUDA.
@@ -157,6 +168,7 @@ int take_check_score(int* out4);
 void set_fault(int extra_peers, unsigned long long wait_limit_ns);
 int take_check_select(int* out4);
 int take_check_compact(int* out4);
+int take_check_leverage(int* out4);
 static __device__ __noinline__ void kvp_check_fail(int code, int a, int b) {
     if (atomicCAS(&g_kvp_check[0], 0, code) == 0) {
         g_kvp_check[1] = a;

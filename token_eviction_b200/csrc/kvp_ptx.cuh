@@ -210,6 +210,30 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Waits for phase `parity` of `bar`, sleeping in the barrier between looks at the clock
+// and at `abort_flag` (shared memory: set when another thread of the CTA gave up). After
+// `limit_ns` the first error `code` goes into `err` (global memory), the abort flag is set
+// and false returned. Out of line: the slow part of every wait, one copy per file.
+static __device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, int* abort_flag,
+                                                      unsigned long long limit_ns, int* err, int code) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+        if (*(volatile int*)abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            atomicCAS(err, 0, code);
+            *(volatile int*)abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// Makes this thread's ordinary (generic-proxy) writes to shared memory visible to the
+// async proxy: operands the tensor cores read through descriptors.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -139,28 +139,14 @@ struct SmemBars {
 // Wait for phase `parity` of `bar`; false if the CTA is unwinding or the wait timed out
 // (then the first error code is recorded and the CTA told to unwind). After the first
 // test the thread sleeps in the barrier (woken by the phase's completion, or after at most
-// kSleepNs to look at the clock), so that waiting warps do not flood shared memory with
+// 20 us to look at the clock), so that waiting warps do not flood shared memory with
 // polls while the TMA, the tensor cores and the working warps use it.
-// The sleeping part is out of line: it is entered only when the first test fails, and
-// one copy of it keeps the kernel's code small.
-constexpr uint32_t kSleepNs = 20000;
-__device__ __noinline__ bool wait_phase_slow(uint64_t* bar, uint32_t parity, int* abort_flag,
-                                             unsigned long long limit_ns, int* err, int code) {
-    const uint64_t t0 = ptx::globaltimer_ns();
-    while (true) {
-        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
-        if (*(volatile int*)abort_flag) return false;
-        if (ptx::globaltimer_ns() - t0 > limit_ns) {
-            atomicCAS(err, 0, code);
-            *(volatile int*)abort_flag = 1;
-            return false;
-        }
-    }
-}
+// The sleeping part is out of line (bounded_wait_slow): it is entered only when the first
+// test fails, and one copy of it keeps the kernel's code small.
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemBars* sb,
                                            const Params& p, int code) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    return wait_phase_slow(bar, parity, &sb->abort_flag, p.wait_limit_ns, p.err, code);
+    return ptx::bounded_wait_slow(bar, parity, &sb->abort_flag, p.wait_limit_ns, p.err, code);
 }
 
 // wait_phase for the roles whose warps work as a whole (S2, epilogue): the warp takes one
@@ -175,7 +161,7 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, SmemBa
 // used before exit, so that no copy or MMA is still writing this CTA's memory.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = ptx::globaltimer_ns();
-    while (!ptx::mbar_try_wait_sleep(bar, parity, kSleepNs))
+    while (!ptx::mbar_try_wait_sleep(bar, parity, 20000))
         if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) return;
 }
 
@@ -343,6 +329,7 @@ __device__ __forceinline__ void v_worker(uint8_t* smem, const Params& p, int n, 
         if (vi >= kS2Ring && !wait_warp(&sb->s2empty[rs], (vi / kS2Ring - 1) & 1, sb, p, kErrWaitS2)) break;
         if (!wait_warp(&sb->vfull[vi % p.nv], (vi / p.nv) & 1, sb, p, kErrWaitS2)) break;
         if (lane == 0 && c % kVPieces == 0) KVP_MSTAMP(vi, 0);
+        if (lane == 0) KVP_MSTAMP(vi, 3 + (int)(c % kVPieces));
         const int key = (int)(c % kVPieces) * kKeys + lane;
         const float s2 = row_absmax<D>(Slots + (p.nk + vi % p.nv) * kSlotBytes + key * (D * 2), lane);
         __syncwarp();                                     // every lane is done with the V slot
@@ -353,6 +340,7 @@ __device__ __forceinline__ void v_worker(uint8_t* smem, const Params& p, int n, 
             __threadfence_block();
             ptx::mbar_arrive(&sb->s2full[rs]);
             if (c % kVPieces == kVPieces - 1) KVP_MSTAMP(vi, 1);
+            KVP_MSTAMP(vi, 7 + (int)(c % kVPieces));
         }
     }
 }
@@ -912,32 +900,6 @@ namespace kvp {
 
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-// bf16 tensor map of `rank` dims (innermost first), tile box `box`.
-bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle swz) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint32_t estride[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
-                    strides_bytes, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 struct Launch {
     Params p;
     int grid;
@@ -1030,6 +992,35 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
 }
 
 }  // namespace
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+}  // namespace
+
+// bf16 tensor map of `rank` dims (innermost first), tile box `box`.
+bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                    strides_bytes, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 cudaError_t launch_score(const kvp_shape& s, const Plan& plan, const uint16_t* q, const uint16_t* k,
                          const uint16_t* v, void* workspace, float* score, float* s1, float* s2,
