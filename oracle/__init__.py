@@ -54,6 +54,8 @@ def _get():
         lib.oracle_select_policy.restype = i
         lib.oracle_leverage.argtypes = [i, i, i, i, p, p, p, p, p, p]
         lib.oracle_leverage.restype = i
+        lib.oracle_select_adaptive.argtypes = [i, i, i, i, i, ctypes.c_double, p, p, p]
+        lib.oracle_select_adaptive.restype = i
         _lib = lib
     return _lib
 
@@ -164,3 +166,18 @@ def oracle_leverage(k, v, g, want_parts: bool = False):
     if rc != 0:
         raise ValueError("oracle_leverage: bad size")
     return (score, lk, lv) if want_parts else score
+
+
+def oracle_select_adaptive(score, window: int, budget: int, alpha: float):
+    """Adaptive per-head budgets (AdaKV, as the CurDKV rebuttal page describes it): score
+    [b, hkv, L]. Returns (idx [b, hkv * B] int32: each head's kept positions, ascending,
+    heads one after another; counts [b, hkv] int32, window included)."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    b, hkv, L = score.shape
+    idx = np.empty((b, hkv * budget), dtype=np.int32)
+    counts = np.empty((b, hkv), dtype=np.int32)
+    rc = _get().oracle_select_adaptive(b, hkv, L, window, budget, float(alpha), score.ctypes.data,
+                                       idx.ctypes.data, counts.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_select_adaptive: bad size or alpha")
+    return idx, counts

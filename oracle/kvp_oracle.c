@@ -44,6 +44,15 @@
  * norms); "combined" is the product lk_j * lv_j (as SlimKV combines S1 and S2); the
  * normalisation divides by the sum over the head's L positions (all zero if that is 0).
  *
+ * Adaptive per-head budgets (oracle_select_adaptive), the AdaKV scheme the CurDKV
+ * rebuttal page describes in "On the sensitivity of the safeguard parameter (alpha)"
+ * (Tables 5-6): the heads of a layer share one budget, and alpha sets the share every head
+ * keeps for itself. Readings: per sequence, each KV head keeps its w window positions
+ * and a floor of f = floor(alpha (B - w)) of its own best candidates (score descending,
+ * then position ascending); the other hkv (B - w - f) positions go to the best of all
+ * heads' remaining candidates (score descending, then head, then position ascending). The
+ * sequence keeps hkv B positions in all, as with a uniform budget.
+ *
  * Parity pins (tests): sum_j S1 = G w; closed forms for identical keys and for a
  * single planted key; G = 1, w = 1 against a library softmax; brute force on tiny
  * inputs; selection against a library stable sort; gather against library indexing;
@@ -292,5 +301,76 @@ int oracle_leverage(int rows, int L, int d, int r, const uint16_t* k, const uint
         for (int j = 0; j < L; ++j) out[j] = total > 0.0 ? out[j] / total : 0.0;
     }
     free(gd);
+    return 0;
+}
+
+typedef struct {
+    double s;
+    int h, j;
+} cand3_t;
+
+static int by_score_head_pos(const void* a, const void* b) {
+    const cand3_t* x = (const cand3_t*)a;
+    const cand3_t* y = (const cand3_t*)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    if (x->h != y->h) return x->h < y->h ? -1 : 1;
+    return x->j < y->j ? -1 : (x->j > y->j);
+}
+
+/*
+ * Adaptive budgets for `batch` sequences of `hkv` KV heads.
+ *   score  [batch][hkv][L]
+ *   counts [batch][hkv]      kept positions of each head (window included)
+ *   idx    [batch][hkv * B]  each head's kept positions, ascending, heads one after another
+ * Returns 0, or -1 on a bad size or alpha outside [0, 1].
+ */
+int oracle_select_adaptive(int batch, int hkv, int L, int w, int B, double alpha,
+                           const double* score, int32_t* idx, int32_t* counts) {
+    if (batch < 0 || hkv < 1 || w < 1 || w > L || B < w || B > L) return -1;
+    if (!(alpha >= 0.0 && alpha <= 1.0)) return -1;
+    const int n = L - w;
+    const int f = (int)floor(alpha * (double)(B - w));
+    const long long R = (long long)hkv * (B - w - f);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < batch; ++b) {
+        unsigned char* keep = (unsigned char*)calloc((size_t)hkv * L, 1);
+        cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)(n > 0 ? n : 1));
+        cand3_t* pool = (cand3_t*)malloc(sizeof(cand3_t) * (size_t)hkv * (n > 0 ? n : 1));
+        long long np = 0;
+        for (int h = 0; h < hkv; ++h) {
+            const double* row = score + ((size_t)b * hkv + h) * L;
+            unsigned char* kr = keep + (size_t)h * L;
+            for (int j = 0; j < n; ++j) {
+                c[j].s = row[j];
+                c[j].j = j;
+            }
+            qsort(c, (size_t)n, sizeof(cand_t), by_score_then_pos);
+            for (int t = 0; t < f; ++t) kr[c[t].j] = 1;          /* the head's floor */
+            for (int t = f; t < n; ++t) {                          /* the rest joins the pool */
+                pool[np].s = c[t].s;
+                pool[np].h = h;
+                pool[np].j = c[t].j;
+                ++np;
+            }
+            for (int j = n; j < L; ++j) kr[j] = 1;                 /* the window */
+        }
+        qsort(pool, (size_t)np, sizeof(cand3_t), by_score_head_pos);
+        for (long long t = 0; t < R && t < np; ++t) keep[(size_t)pool[t].h * L + pool[t].j] = 1;
+        int32_t* out = idx + (size_t)b * hkv * B;
+        long long o = 0;
+        for (int h = 0; h < hkv; ++h) {
+            int cnt = 0;
+            for (int j = 0; j < L; ++j)
+                if (keep[(size_t)h * L + j]) {
+                    out[o++] = j;
+                    ++cnt;
+                }
+            counts[(size_t)b * hkv + h] = cnt;
+        }
+        free(pool);
+        free(c);
+        free(keep);
+    }
     return 0;
 }

@@ -429,3 +429,92 @@ def test_leverage_invariants():
     kz = k.copy()
     kz[1, 17] = 0
     assert oracle.oracle_leverage(kz, v, g)[1, 17] == 0.0
+
+
+# ---- AdaKV adaptive budgets (CurDKV rebuttal page, "On the sensitivity of the safeguard
+#      parameter (alpha)", Tables 5-6)
+
+def unpack(idx, counts, b, h):
+    off = int(counts[b, :h].sum())
+    return idx[b, off:off + counts[b, h]]
+
+
+def adaptive_inputs(b, hkv, L, seed):
+    rng = np.random.default_rng(seed)
+    s = rng.random((b, hkv, L)) ** 3 * rng.uniform(0.2, 5.0, (b, hkv, 1))
+    s[:, :, 5:40] = np.round(s[:, :, 5:40], 1)        # a block of ties within and across heads
+    return s
+
+
+def test_adaptive_alpha_one_is_the_uniform_budget():
+    """alpha = 1: every head keeps its own best B - w and the window (numpy's stable sort)."""
+    b, hkv, L, w, B = 2, 3, 300, 8, 60
+    s = adaptive_inputs(b, hkv, L, 21)
+    idx, counts = oracle.oracle_select_adaptive(s, w, B, 1.0)
+    assert (counts == B).all()
+    for bi in range(b):
+        for h in range(hkv):
+            np.testing.assert_array_equal(unpack(idx, counts, bi, h), library_select(s[bi, h], w, B))
+
+
+def test_adaptive_alpha_zero_is_one_global_top_k():
+    """alpha = 0: the sequence's hkv (B - w) non-window positions are the best of all its
+    heads' candidates, ordered by (score desc, head, position) with numpy's lexsort."""
+    b, hkv, L, w, B = 2, 4, 200, 5, 40
+    s = adaptive_inputs(b, hkv, L, 22)
+    idx, counts = oracle.oracle_select_adaptive(s, w, B, 0.0)
+    n = L - w
+    for bi in range(b):
+        hh, jj = np.meshgrid(np.arange(hkv), np.arange(n), indexing="ij")
+        sc = s[bi, :, :n]
+        order = np.lexsort((jj.ravel(), hh.ravel(), -sc.ravel()))[: hkv * (B - w)]
+        keep = np.zeros((hkv, L), bool)
+        keep[hh.ravel()[order], jj.ravel()[order]] = True
+        keep[:, n:] = True
+        for h in range(hkv):
+            np.testing.assert_array_equal(unpack(idx, counts, bi, h), np.flatnonzero(keep[h]))
+
+
+@pytest.mark.parametrize("alpha", [0.2, 0.5, 0.9])
+def test_adaptive_exchange_property(alpha):
+    """Any alpha: each head keeps its window and at least its best floor(alpha (B - w));
+    the sequence keeps hkv B in all; and no unkept candidate outranks a kept one that is
+    not in its head's floor (in (score desc, head, position) order)."""
+    b, hkv, L, w, B = 2, 5, 400, 16, 80
+    s = adaptive_inputs(b, hkv, L, 23)
+    idx, counts = oracle.oracle_select_adaptive(s, w, B, alpha)
+    n, f = L - w, int(np.floor(alpha * (B - w)))
+    assert (counts.sum(1) == hkv * B).all()
+    for bi in range(b):
+        kept_extra, unkept = [], []
+        for h in range(hkv):
+            kept = unpack(idx, counts, bi, h)
+            assert (np.diff(kept) > 0).all()
+            assert set(range(n, L)) <= set(kept.tolist())
+            floor = library_select(s[bi, h], w, f + w)[:f]
+            assert set(floor.tolist()) <= set(kept.tolist())
+            others = set(kept.tolist()) - set(floor.tolist()) - set(range(n, L))
+            kept_extra += [(-s[bi, h, j], h, j) for j in others]
+            unkept += [(-s[bi, h, j], h, j) for j in set(range(n)) - set(kept.tolist())]
+        if kept_extra and unkept:
+            assert max(kept_extra) < min(unkept)
+
+
+def test_adaptive_equal_scores_fill_the_lowest_heads_first():
+    """All scores equal, alpha = 0: the shared positions go to head 0's candidates in
+    position order, then head 1's, ... (the tie rule), a closed form."""
+    hkv, L, w, B = 3, 50, 4, 20
+    s = np.ones((1, hkv, L))
+    idx, counts = oracle.oracle_select_adaptive(s, w, B, 0.0)
+    n, R = L - w, hkv * (B - w)
+    expect = []
+    for h in range(hkv):
+        take = max(0, min(n, R - h * n))
+        expect.append(np.concatenate([np.arange(take), np.arange(n, L)]))
+    np.testing.assert_array_equal(counts[0], [len(e) for e in expect])
+    np.testing.assert_array_equal(idx[0], np.concatenate(expect))
+
+
+def test_adaptive_rejects_bad_alpha():
+    with pytest.raises(ValueError):
+        oracle.oracle_select_adaptive(np.ones((1, 2, 10)), 2, 5, 1.5)
