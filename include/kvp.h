@@ -154,6 +154,38 @@ KVP_API kvp_status kvp_leverage(const kvp_shape* shape, const uint16_t* k, const
                                 size_t workspace_bytes, void* stream);
 
 /*
+ * Adaptive per-head budgets: the AdaKV scheme with its safeguard alpha, as the CurDKV
+ * rebuttal page describes it ("On the sensitivity of the safeguard parameter (alpha)",
+ * Tables 5-6; the AdaKV default alpha is 0.20). The KV heads of a sequence share its
+ * budget hkv * B. Every head keeps its window [L - w, L) and its best
+ * f = floor(alpha * (B - w)) candidates of [0, L - w) (score descending, then position);
+ * the other hkv * (B - w - f) positions go to the best of all the heads' remaining
+ * candidates (score descending, then head, then position). alpha = 1 is kvp_select's
+ * uniform budget; alpha = 0 one shared top-k.
+ *   score   [b, hkv, L] fp32, non-negative (kvp_score's S, or kvp_leverage's)
+ *   idx     [b, hkv * B] int32 output: head 0's kept positions ascending, then head 1's, ...
+ *   counts  [b, hkv] int32 output: kept positions of each head (window included); they sum
+ *           to hkv * B per sequence
+ *   workspace  at least kvp_adaptive_workspace_bytes(shape) bytes (0 for a bad shape)
+ * Needs 0 <= alpha <= 1 and hkv <= 4096 (else KVP_ERR_SHAPE).
+ */
+KVP_API size_t kvp_adaptive_workspace_bytes(const kvp_shape* shape);
+KVP_API kvp_status kvp_select_adaptive(const kvp_shape* shape, float alpha, const float* score,
+                                       int32_t* idx, int32_t* counts, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
+ * Compaction of a ragged selection (kvp_select_adaptive's layout): row r of sequence b's
+ * output belongs to the head h whose rows [sum of counts[b, :h], + counts[b, h]) hold it,
+ * and k_out[b, r, :] = k[b, h, idx[b, r], :]; the same for v; a bit copy.
+ *   idx     [b, hkv * B] int32;  counts [b, hkv] int32 (summing to hkv * B)
+ *   k_out, v_out  [b, hkv * B, d] bf16 outputs; an index outside [0, L) yields a zero row
+ */
+KVP_API kvp_status kvp_compact_ragged(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
+                                      const int32_t* idx, const int32_t* counts, uint16_t* k_out,
+                                      uint16_t* v_out, void* stream);
+
+/*
  * Compaction: k_out[b, h, t, :] = k[b, h, idx[b, h, t], :], the same for v; a bit copy.
  *   k, v          [b, hkv, L, d] bf16
  *   idx           [b, hkv, B]    int32, entries in [0, L) (an entry outside that range

@@ -20,7 +20,7 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     assert {"kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_select_policy", "kvp_compact",
-            "kvp_workspace_status",
+            "kvp_leverage", "kvp_select_adaptive", "kvp_compact_ragged", "kvp_workspace_status",
             "kvp_score_static", "kvp_score_static_status", "kvp_status_string",
             "kvp_last_cuda_error"} <= declared_symbols()
 
@@ -112,6 +112,23 @@ def test_policy_select_rejects_bad_policies_on_the_host():
     assert call(mode=2, s2=None) == 1
     assert call(s1=24) == 3                   # misaligned
     assert m._lib.kvp_select_policy(ctypes.byref(sh), None, 16, 16, 16, None) == 1
+
+
+def test_adaptive_calls_reject_bad_arguments_on_the_host():
+    import token_eviction_b200 as m
+    sh = m.make_shape(1, 32, 8, 128, 4096, 32, 256)
+    lib = m._lib
+    ws_bytes = lib.kvp_adaptive_workspace_bytes(ctypes.byref(sh))
+    assert ws_bytes >= 8 * 4096 * 4
+    assert lib.kvp_adaptive_workspace_bytes(ctypes.byref(m.make_shape(1, 32, 8, 100, 4096, 32, 256))) == 0
+    sel = lib.kvp_select_adaptive
+    assert sel(ctypes.byref(sh), ctypes.c_float(1.5), 16, 16, 16, 16, ws_bytes, None) == 2
+    assert sel(ctypes.byref(sh), ctypes.c_float(float("nan")), 16, 16, 16, 16, ws_bytes, None) == 2
+    assert sel(ctypes.byref(sh), ctypes.c_float(0.2), 16, None, 16, 16, ws_bytes, None) == 1
+    assert sel(ctypes.byref(sh), ctypes.c_float(0.2), 16, 16, 16, 16, 8, None) == 4
+    assert sel(ctypes.byref(sh), ctypes.c_float(0.2), 16, 16, 20, 16, ws_bytes, None) == 3
+    assert lib.kvp_compact_ragged(ctypes.byref(sh), 16, 16, 16, None, 16, 16, None) == 1
+    assert lib.kvp_compact_ragged(ctypes.byref(sh), 16, 16, 16, 16, 16, 8, None) == 3
 
 
 def test_binding_validates_tensors_before_calling():

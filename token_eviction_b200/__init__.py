@@ -12,6 +12,8 @@ The functions carry the C names:
 * ``kvp_select(shape, score, idx, workspace=None, stream=None)``
 * ``kvp_select_policy(shape, policy, s1, s2, idx, stream=None)``
 * ``kvp_leverage(shape, k, v, g, score, workspace=None, stream=None)``
+* ``kvp_select_adaptive(shape, alpha, score, idx, counts, workspace=None, stream=None)``
+* ``kvp_compact_ragged(shape, k, v, idx, counts, k_out, v_out, stream=None)``
 * ``kvp_compact(shape, k, v, idx, k_out, v_out, stream=None)``
 * ``kvp_workspace_status(workspace, stream=None)``
 * ``kvp_status_string(status)``
@@ -87,6 +89,12 @@ def _load():
     lib.kvp_select_policy.restype = ctypes.c_int
     lib.kvp_leverage.argtypes = [S, P, P, P, ctypes.c_int32, P, P, ctypes.c_size_t, P]
     lib.kvp_leverage.restype = ctypes.c_int
+    lib.kvp_adaptive_workspace_bytes.argtypes = [S]
+    lib.kvp_adaptive_workspace_bytes.restype = ctypes.c_size_t
+    lib.kvp_select_adaptive.argtypes = [S, ctypes.c_float, P, P, P, P, ctypes.c_size_t, P]
+    lib.kvp_select_adaptive.restype = ctypes.c_int
+    lib.kvp_compact_ragged.argtypes = [S, P, P, P, P, P, P, P]
+    lib.kvp_compact_ragged.restype = ctypes.c_int
     lib.kvp_compact.argtypes = [S, P, P, P, P, P, P]
     lib.kvp_compact.restype = ctypes.c_int
     lib.kvp_status_string.argtypes = [ctypes.c_int]
@@ -110,7 +118,7 @@ _lib = _load()
 KERNELS_PER_LAYER = 3
 
 EXPORTED = ("kvp_workspace_bytes", "kvp_score", "kvp_select", "kvp_select_policy", "kvp_leverage",
-            "kvp_compact",
+            "kvp_adaptive_workspace_bytes", "kvp_select_adaptive", "kvp_compact_ragged", "kvp_compact",
             "kvp_workspace_status",
             "kvp_score_static", "kvp_score_static_status", "kvp_status_string", "kvp_last_cuda_error")
 
@@ -240,6 +248,39 @@ def kvp_leverage(shape, k, v, g, score, workspace=None, stream=None):
                            workspace.numel(), _stream(stream))
     if st != KVP_OK:
         raise KvpError(st, "kvp_leverage")
+
+
+def kvp_select_adaptive(shape, alpha, score, idx, counts, workspace=None, stream=None):
+    """Adaptive per-head budgets (AdaKV with safeguard alpha): idx [b, hkv * B] packed
+    head after head, counts [b, hkv]."""
+    sh = _as_shape(shape)
+    b, hkv, L, B = sh.batch, sh.hkv, sh.seq_len, sh.budget
+    ps = _ptr(score, "score", torch.float32, (b, hkv, L))
+    pi = _ptr(idx, "idx", torch.int32, (b, hkv * B))
+    pc = _ptr(counts, "counts", torch.int32, (b, hkv))
+    if workspace is None:
+        n = int(_lib.kvp_adaptive_workspace_bytes(ctypes.byref(sh)))
+        if n == 0:
+            raise KvpError(2, "kvp_adaptive_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=score.device)
+    st = _lib.kvp_select_adaptive(ctypes.byref(sh), float(alpha), ps, pi, pc, workspace.data_ptr(),
+                                  workspace.numel(), _stream(stream))
+    if st != KVP_OK:
+        raise KvpError(st, "kvp_select_adaptive")
+
+
+def kvp_compact_ragged(shape, k, v, idx, counts, k_out, v_out, stream=None):
+    sh = _as_shape(shape)
+    b, hkv, d, L, B = sh.batch, sh.hkv, sh.head_dim, sh.seq_len, sh.budget
+    args = (_ptr(k, "k", torch.bfloat16, (b, hkv, L, d)),
+            _ptr(v, "v", torch.bfloat16, (b, hkv, L, d)),
+            _ptr(idx, "idx", torch.int32, (b, hkv * B)),
+            _ptr(counts, "counts", torch.int32, (b, hkv)),
+            _ptr(k_out, "k_out", torch.bfloat16, (b, hkv * B, d)),
+            _ptr(v_out, "v_out", torch.bfloat16, (b, hkv * B, d)))
+    st = _lib.kvp_compact_ragged(ctypes.byref(sh), *args, _stream(stream))
+    if st != KVP_OK:
+        raise KvpError(st, "kvp_compact_ragged")
 
 
 def kvp_compact(shape, k, v, idx, k_out, v_out, stream=None):

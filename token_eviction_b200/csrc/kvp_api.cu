@@ -150,6 +150,46 @@ extern "C" kvp_status kvp_leverage(const kvp_shape* shape, const uint16_t* k, co
     return KVP_OK;
 }
 
+// KV heads per sequence that the adaptive calls accept (their offsets sit in shared memory)
+static constexpr int kMaxAdaptiveHeads = 4096;
+
+extern "C" size_t kvp_adaptive_workspace_bytes(const kvp_shape* shape) {
+    Plan p;
+    if (!shape || !plan_of(*shape, &p) || shape->hkv > kMaxAdaptiveHeads) return 0;
+    return adaptive_workspace_bytes(*shape);
+}
+
+extern "C" kvp_status kvp_select_adaptive(const kvp_shape* shape, float alpha, const float* score,
+                                          int32_t* idx, int32_t* counts, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+    if (!shape || !score || !idx || !counts) return KVP_ERR_NULL;
+    Plan p;
+    if (!plan_of(*shape, &p) || shape->hkv > kMaxAdaptiveHeads) return KVP_ERR_SHAPE;
+    if (!(alpha >= 0.f && alpha <= 1.f)) return KVP_ERR_SHAPE;
+    if (!aligned16(score) || !aligned16(idx) || !aligned16(counts)) return KVP_ERR_ALIGN;
+    if (!workspace || workspace_bytes < adaptive_workspace_bytes(*shape)) return KVP_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KVP_ERR_ALIGN;
+    const cudaError_t e =
+        launch_select_adaptive(*shape, alpha, score, idx, counts, workspace, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_failed(e);
+    return KVP_OK;
+}
+
+extern "C" kvp_status kvp_compact_ragged(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
+                                         const int32_t* idx, const int32_t* counts, uint16_t* k_out,
+                                         uint16_t* v_out, void* stream) {
+    if (!shape || !k || !v || !idx || !counts || !k_out || !v_out) return KVP_ERR_NULL;
+    Plan p;
+    if (!plan_of(*shape, &p) || shape->hkv > kMaxAdaptiveHeads) return KVP_ERR_SHAPE;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(counts) || !aligned16(k_out) ||
+        !aligned16(v_out))
+        return KVP_ERR_ALIGN;
+    const cudaError_t e =
+        launch_compact_ragged(*shape, k, v, idx, counts, k_out, v_out, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_failed(e);
+    return KVP_OK;
+}
+
 extern "C" kvp_status kvp_compact(const kvp_shape* shape, const uint16_t* k, const uint16_t* v,
                                   const int32_t* idx, uint16_t* k_out, uint16_t* v_out,
                                   void* stream) {
@@ -179,15 +219,15 @@ extern "C" KVP_API void kvp_debug_set_fault(int extra_peers, unsigned long long 
 
 // Debug builds only: copy out (and clear) the first failed device-side bounds check.
 extern "C" KVP_API int kvp_debug_take_check_unit(int unit, int* out4) {
-    int (*readers[4])(int*) = {take_check_score, take_check_select, take_check_compact,
-                               take_check_leverage};
-    if (unit < 0 || unit > 3) return -1;
+    int (*readers[5])(int*) = {take_check_score, take_check_select, take_check_compact,
+                               take_check_leverage, take_check_adaptive};
+    if (unit < 0 || unit > 4) return -1;
     return readers[unit](out4);
 }
 
 extern "C" KVP_API int kvp_debug_take_check(int* out4) {
-    int (*readers[4])(int*) = {take_check_score, take_check_select, take_check_compact,
-                               take_check_leverage};
+    int (*readers[5])(int*) = {take_check_score, take_check_select, take_check_compact,
+                               take_check_leverage, take_check_adaptive};
     out4[0] = out4[1] = out4[2] = out4[3] = 0;
     for (auto rd : readers) {
         int v[4];

@@ -130,6 +130,14 @@ cudaError_t launch_leverage(const kvp_shape& s, const Plan& p, const uint16_t* k
 // Bytes of the leverage kernel's partial sums with `grid` CTAs (they live in the
 // workspace's partial-softmax region) and the slots per KV head.
 size_t leverage_part_bytes(const kvp_shape& s, const Plan& p, int grid, int* maxparts);
+// Adaptive per-head budgets (kvp_adaptive.cu).
+size_t adaptive_workspace_bytes(const kvp_shape& s);
+int adaptive_floor(const kvp_shape& s, float alpha);
+cudaError_t launch_select_adaptive(const kvp_shape& s, float alpha, const float* score, int32_t* idx,
+                                   int32_t* counts, void* workspace, cudaStream_t st);
+cudaError_t launch_compact_ragged(const kvp_shape& s, const uint16_t* k, const uint16_t* v,
+                                  const int32_t* idx, const int32_t* counts, uint16_t* k_out,
+                                  uint16_t* v_out, cudaStream_t st);
 cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t* v,
                            const int32_t* idx, uint16_t* k_out, uint16_t* v_out, cudaStream_t st);
 
@@ -169,6 +177,7 @@ void set_fault(int extra_peers, unsigned long long wait_limit_ns);
 int take_check_select(int* out4);
 int take_check_compact(int* out4);
 int take_check_leverage(int* out4);
+int take_check_adaptive(int* out4);
 static __device__ __noinline__ void kvp_check_fail(int code, int a, int b) {
     if (atomicCAS(&g_kvp_check[0], 0, code) == 0) {
         g_kvp_check[1] = a;

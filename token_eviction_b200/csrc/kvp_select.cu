@@ -286,13 +286,15 @@ select_cluster(const SelSource src, int32_t* __restrict__ idx, int L, int w, int
 
 namespace {
 
-cudaError_t launch_select_source(const kvp_shape& s, const SelSource& src, int32_t* idx, cudaStream_t st) {
-    const int nc = s.seq_len - s.window - src.sinks;      // candidates
+// rows rows of L scores each: candidates [sinks, L - w), budget B (window and sinks included)
+cudaError_t launch_select_source(int rows, int L, int w, int B, const SelSource& src, int32_t* idx,
+                                 cudaStream_t st) {
+    const int nc = L - w - src.sinks;                     // candidates
     const int slice = (nc + kCl - 1) / kCl;
     const bool in_smem = slice <= kSliceCap;
     const size_t dyn = in_smem ? (size_t)slice * sizeof(uint32_t) : 0;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(s.batch * s.hkv * kCl);
+    cfg.gridDim = dim3(rows * kCl);
     cfg.blockDim = dim3(kSelThreads);
     cfg.dynamicSmemBytes = dyn;
     cfg.stream = st;
@@ -306,25 +308,31 @@ cudaError_t launch_select_source(const kvp_shape& s, const SelSource& src, int32
     cudaError_t e;
     if (in_smem) {
         if ((e = allow_dynamic_smem((const void*)select_cluster<true>, dyn)) != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, select_cluster<true>, src, idx, s.seq_len, s.window, s.budget, slice);
+        return cudaLaunchKernelEx(&cfg, select_cluster<true>, src, idx, L, w, B, slice);
     }
-    return cudaLaunchKernelEx(&cfg, select_cluster<false>, src, idx, s.seq_len, s.window, s.budget, slice);
+    return cudaLaunchKernelEx(&cfg, select_cluster<false>, src, idx, L, w, B, slice);
 }
 
 }  // namespace
+
+cudaError_t launch_select_rows(int rows, int L, int w, int B, const float* score, int32_t* idx,
+                               cudaStream_t st) {
+    const SelSource src = {score, nullptr, nullptr, 0, 1, 0};
+    return launch_select_source(rows, L, w, B, src, idx, st);
+}
 
 cudaError_t launch_select(const kvp_shape& s, const Plan& p, const float* score, int32_t* idx,
                           void* scratch, cudaStream_t st) {
     (void)p;
     (void)scratch;
     const SelSource src = {score, nullptr, nullptr, 0, 1, 0};
-    return launch_select_source(s, src, idx, st);
+    return launch_select_source(s.batch * s.hkv, s.seq_len, s.window, s.budget, src, idx, st);
 }
 
 cudaError_t launch_select_policy(const kvp_shape& s, const kvp_policy& pol, const float* s1,
                                  const float* s2, int32_t* idx, cudaStream_t st) {
     const SelSource src = {nullptr, s1, s2, pol.sinks, pol.pool_kernel, pol.mode};
-    return launch_select_source(s, src, idx, st);
+    return launch_select_source(s.batch * s.hkv, s.seq_len, s.window, s.budget, src, idx, st);
 }
 
 #ifdef KVP_CHECKS
