@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="kvp", choices=["kvp", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-paths", action="store_true",
+                    help="skip the per-call timing of the policy/adaptive selections and the "
+                         "leverage scorer")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every call from the host instead of replaying CUDA graphs")
     a = ap.parse_args()
@@ -252,6 +255,63 @@ def workload_config(wl, l2_note):
             "budget": wl.budget, "layers_per_step": 1, "l2": l2_note}
 
 
+def measure_extra_paths(kvp, torch, sh, wl, sets, bufs, dev, stream, peak, n=40):
+    """Per-call device times (CUDA events on the launching stream, median of n calls after
+    warm-up, outside the timed region) of the calls beside the headline path, on the same
+    workload: the policy selection (sinks, S1 pooling), the CurDKV leverage scorer (r = 20,
+    rotating input sets larger than L2), the adaptive per-head budgets (alpha = 0.20) and
+    the ragged compaction."""
+    b, hkv, L, d, B = wl.batch, wl.hkv, wl.seq_len, wl.head_dim, wl.budget
+    buf = bufs[0]
+    q, k, v = sets[0]
+    s1 = torch.empty((b, hkv, L), dtype=torch.float32, device=dev)
+    s2 = torch.empty_like(s1)
+    kvp.kvp_score(sh, q, k, v, buf.score, s1, s2, buf.workspace, stream)
+    g = torch.from_numpy(synth.normal_bf16(d, 20, 99, 3).view(np.int16)).view(torch.bfloat16).to(dev)
+    lev = torch.empty_like(s1)
+    idx = torch.empty((b, hkv, B), dtype=torch.int32, device=dev)
+    aidx = torch.empty((b, hkv * B), dtype=torch.int32, device=dev)
+    counts = torch.empty((b, hkv), dtype=torch.int32, device=dev)
+    aws = kvp.adaptive_workspace_for(sh, dev)
+    k_out = torch.empty((b, hkv * B, d), dtype=torch.bfloat16, device=dev)
+    v_out = torch.empty_like(k_out)
+    pol = kvp.make_policy(4, 7, kvp.RANK_PRODUCT)
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize(dev)
+        ts = []
+        for i in range(n):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(i)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        return float(np.median(ts))
+
+    nsets = len(sets)
+    t_pol = timed(lambda i: kvp.kvp_select_policy(sh, pol, s1, s2, idx, stream))
+    t_lev = timed(lambda i: kvp.kvp_leverage(sh, sets[i % nsets][1], sets[i % nsets][2], g, lev,
+                                             bufs[i % nsets].workspace, stream))
+    t_ada = timed(lambda i: kvp.kvp_select_adaptive(sh, 0.2, buf.score, aidx, counts, aws, stream))
+    t_rag = timed(lambda i: kvp.kvp_compact_ragged(sh, sets[i % nsets][1], sets[i % nsets][2], aidx,
+                                                   counts, k_out, v_out, stream))
+    lev_bytes = 2 * b * hkv * L * d * 2 + b * hkv * L * 4 * 3          # K, V; score written, scaled
+    rag_bytes = 2 * 2 * b * hkv * B * d * 2 + b * hkv * B * 4          # rows read + written; idx
+    return {
+        "kvp_select_policy": {"ms": t_pol, "policy": "sinks 4, S1 max-pool kernel 7, pool(S1)*S2"},
+        "kvp_leverage": {"ms": t_lev, "r": 20, "algorithmic_bytes": lev_bytes,
+                         "achieved_gbs": lev_bytes / (t_lev * 1e-3) / 1e9,
+                         "frac": lev_bytes / (t_lev * 1e-3) / 1e9 / peak},
+        "kvp_select_adaptive": {"ms": t_ada, "alpha": 0.2},
+        "kvp_compact_ragged": {"ms": t_rag, "algorithmic_bytes": rag_bytes,
+                               "achieved_gbs": rag_bytes / (t_rag * 1e-3) / 1e9,
+                               "frac": rag_bytes / (t_rag * 1e-3) / 1e9 / peak},
+    }
+
+
 def run_kvp(a, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -397,9 +457,11 @@ def run_kvp(a, world, rank, local):
     idx_np = h_idx.numpy()
     assert (idx_np[..., wl.budget - wl.window:] == np.arange(wl.seq_len - wl.window, wl.seq_len)).all()
 
+    peak, peak_kind = measured_peaks()
+    extra = None if a.no_extra_paths else measure_extra_paths(kvp, torch, sh, wl, sets, bufs, dev, stream, peak)
+
     line = None
     if rank == 0:
-        peak, peak_kind = measured_peaks()
         ms_per_layer = job_ms_per_layer(elapsed_ms, a.steps, world)
         bytes_layer = wl.bytes_per_layer()
         score_bytes = bytes_layer["score"]
@@ -424,6 +486,7 @@ def run_kvp(a, world, rank, local):
             "e2e": {"value": job_ms_per_layer(e2e_ms, e2e_steps, world), "unit": "ms/layer",
                     "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": a.steps * kvp.KERNELS_PER_LAYER,
+            "extra_paths": extra,
             "clocks": clocks.summary(),
         }
         if world == 1 and not a.no_cpu_baseline:

@@ -250,6 +250,13 @@ def kvp_leverage(shape, k, v, g, score, workspace=None, stream=None):
         raise KvpError(st, "kvp_leverage")
 
 
+def adaptive_workspace_for(shape, device=None) -> torch.Tensor:
+    n = int(_lib.kvp_adaptive_workspace_bytes(ctypes.byref(_as_shape(shape))))
+    if n == 0:
+        raise KvpError(2, "kvp_adaptive_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
 def kvp_select_adaptive(shape, alpha, score, idx, counts, workspace=None, stream=None):
     """Adaptive per-head budgets (AdaKV with safeguard alpha): idx [b, hkv * B] packed
     head after head, counts [b, hkv]."""
@@ -259,10 +266,7 @@ def kvp_select_adaptive(shape, alpha, score, idx, counts, workspace=None, stream
     pi = _ptr(idx, "idx", torch.int32, (b, hkv * B))
     pc = _ptr(counts, "counts", torch.int32, (b, hkv))
     if workspace is None:
-        n = int(_lib.kvp_adaptive_workspace_bytes(ctypes.byref(sh)))
-        if n == 0:
-            raise KvpError(2, "kvp_adaptive_workspace_bytes")
-        workspace = torch.empty(n, dtype=torch.uint8, device=score.device)
+        workspace = adaptive_workspace_for(sh, score.device)
     st = _lib.kvp_select_adaptive(ctypes.byref(sh), float(alpha), ps, pi, pc, workspace.data_ptr(),
                                   workspace.numel(), _stream(stream))
     if st != KVP_OK:

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include "kvp_internal.cuh"
+#include "kvp_ptx.cuh"
 
 namespace kvp {
 namespace {
@@ -22,6 +23,7 @@ __global__ void __launch_bounds__(kThreads) gather_rows(const uint4* __restrict_
                                                         uint4* __restrict__ k_out,
                                                         uint4* __restrict__ v_out, int L, int B,
                                                         int piece_shift, int items, int rows_total) {
+    ptx::grid_dependency_wait();         // the indices' producer has completed
     const int stride = gridDim.x * blockDim.x;
     const int pmask = (1 << piece_shift) - 1;
     for (int it = blockIdx.x * blockDim.x + threadIdx.x; it < items; it += stride) {
@@ -58,11 +60,19 @@ cudaError_t launch_compact(const kvp_shape& s, const uint16_t* k, const uint16_t
     if (total > INT32_MAX) return cudaErrorInvalidValue;
     const long long items = total / kPiecesPerThread;
     const long long want = (items + kThreads - 1) / kThreads;
-    const long long cap = (long long)num_sms() * 8;  // 8 resident CTAs of 256 threads per SM
+    // whole waves over the SMs (8 resident CTAs of 256 threads each), so that no SM
+    // carries a second round of CTAs while the others idle
+    const long long sms = num_sms(), cap = sms * 8;
+    const long long grid = want < cap ? (want + sms - 1) / sms * sms : cap;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(want < cap ? want : cap));
+    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
     cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlaps the launch
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     // launched with cudaLaunchKernelEx: its return value is this launch's own error, never
     // a sticky error left by an earlier, unrelated launch
     return cudaLaunchKernelEx(&cfg, gather_rows, (const uint4*)k, (const uint4*)v, idx, (uint4*)k_out,

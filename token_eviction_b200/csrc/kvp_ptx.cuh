@@ -228,6 +228,12 @@ static __device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t pa
     }
 }
 
+// Programmatic dependent launch: wait until the grid this one depends on has completed
+// and its memory is visible (a no-op for a grid launched without the dependency).
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Makes this thread's ordinary (generic-proxy) writes to shared memory visible to the
 // async proxy: operands the tensor cores read through descriptors.
 __device__ __forceinline__ void fence_proxy_async_smem() {

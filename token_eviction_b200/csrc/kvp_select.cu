@@ -23,6 +23,7 @@
 #include <cuda_runtime.h>
 
 #include "kvp_internal.cuh"
+#include "kvp_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -122,6 +123,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 select_cluster(const SelSource src, int32_t* __restrict__ idx, int L, int w, int B, int slice) {
     extern __shared__ uint32_t keys[];   // [slice] when kInSmem
     __shared__ SelShared sh;
+    ptx::grid_dependency_wait();         // the scores' producer has completed
     cg::cluster_group cluster = cg::this_cluster();
     const unsigned rank = cluster.block_rank();
     const int row = blockIdx.x / kCl;
@@ -298,13 +300,17 @@ cudaError_t launch_select_source(int rows, int L, int w, int B, const SelSource&
     cfg.blockDim = dim3(kSelThreads);
     cfg.dynamicSmemBytes = dyn;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kCl;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // launched as a programmatic dependent: its launch overlaps the producer's tail, and
+    // every CTA waits for the producer (grid_dependency_wait) before reading
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t e;
     if (in_smem) {
         if ((e = allow_dynamic_smem((const void*)select_cluster<true>, dyn)) != cudaSuccess) return e;
