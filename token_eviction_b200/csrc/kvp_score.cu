@@ -25,14 +25,16 @@
 //     per row. Per tile each thread sums 2^(t - lse2) over its key's query rows: S1.
 //   S2 comes from phase 1's V tiles (V streams from HBM beside phase 1's K, which comes
 //     mostly from L2: phase 0 streams K alone, so that K stays in L2). Each V tile is cut
-//     into 4 pieces of 32 keys; any warp that would otherwise wait claims the next piece
-//     (in order, through a shared counter) and reduces it into a ring of per-tile S2 rows
-//     in shared memory, which the tile's finishing warps read. No busy warp holds up the V
-//     stream, and the exponentials never wait for V.
+//     into 4 pieces of 32 keys; warps 2 and 3 claim the next piece (in order, through a
+//     shared counter) and reduce it into a ring of per-tile S2 rows in shared memory, which
+//     the tile's finishing warps read. No busy warp holds up the V stream.
+// Query rows: a CTA has at most a few runs of one head each (two with the head-aligned
+// cut); when shared memory allows, every run's query block stays resident (two blocks), so
+// that neither a change of head nor the phase boundary waits for query rows to load again.
 // Warp roles: warp 0 issues the TMA loads (a ring of tile slots in shared memory, and the
 // group's query rows); warp 1 allocates TMEM and issues the MMAs from one thread; warp 2
 // combines the epilogue groups' phase 0 sums and publishes them (so that no epilogue thread
-// waits on a global fence); warp 3 only reduces V pieces; four epilogue warpgroups (warps
+// waits on a global fence), then reduces V pieces like warp 3; four epilogue warpgroups (warps
 // 4-19, one TMEM lane quarter per warp) read the accumulators. TMEM holds four accumulator
 // stages of 128 columns, stage s belonging to epilogue group s. A tile's work is cut into
 // units of at most 128 columns (phase 0: a run of keys over every row block; phase 1: a
@@ -73,27 +75,36 @@ constexpr int kS2Ring = 8;                        // per-tile S2 rows in shared 
 constexpr int kVPieces = 4;                       // pieces of 32 keys per V tile
 constexpr int kMaxParts = 4;                      // phase 1 parts per tile (512 rows / 128)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s on any single wait
+#ifdef KVP_TRACE
+constexpr int kSmemLimit = 227 * 1024 - 10240;   // the trace's static shared arrays take 10 KB
+#else
 constexpr int kSmemLimit = 227 * 1024;
+#endif
 constexpr int kMinSmem = 116 * 1024;              // forces one CTA per SM (TMEM is taken whole)
 constexpr int kQBoxRows = 64;
-constexpr size_t kBarBytes = 640;                 // shared memory reserved for SmemBars
+constexpr size_t kBarBytes = 704;                 // shared memory reserved for SmemBars
+#ifndef KVP_MAX_QBUFS
+#define KVP_MAX_QBUFS 2
+#endif
+constexpr int kMaxQBufs = KVP_MAX_QBUFS;          // resident query blocks (one per run of a head)
 constexpr float kSumLimit = 1.8446744e19f;        // 2^64: a chunk sum above it raises the offset
 
 #ifdef KVP_TRACE
 // Debug builds only: %globaltimer stamps per CTA at phase boundaries.
-// [cta][0..7]: phase boundaries; [8]: SM id; [9]: S2 warps done
+// [cta][0..7]: phase boundaries; [8]: SM id
 __device__ unsigned long long g_kvp_trace[kPlanGrid][12];
 #define KVP_STAMP(i) (g_kvp_trace[blockIdx.x][(i)] = ptx::globaltimer_ns())
-// per-tile events of four CTAs: [cta][tile][event]
+// per-tile events of four CTAs, [cta][tile][event]: kept in shared memory while the kernel
+// runs (no global stores or fences in the traced roles) and copied out at the end
 __device__ unsigned long long g_kvp_ttrace[4][64][8];
 __device__ unsigned long long g_kvp_mtrace[4][64][12];
-#define KVP_MSTAMP(t, e) \
-    ((kvp_trace_slot() >= 0 && (t) < 64) ? (void)(g_kvp_mtrace[kvp_trace_slot()][(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
+__shared__ unsigned long long s_kvp_ttrace[64][8];
+__shared__ unsigned long long s_kvp_mtrace[64][12];
+#define KVP_MSTAMP(t, e) ((t) < 64 ? (void)(s_kvp_mtrace[(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
 __device__ __forceinline__ int kvp_trace_slot() {
     return blockIdx.x == 0 ? 0 : blockIdx.x == 18 ? 1 : blockIdx.x == 73 ? 2 : blockIdx.x == 143 ? 3 : -1;
 }
-#define KVP_TSTAMP(t, e) \
-    ((kvp_trace_slot() >= 0 && (t) < 64) ? (void)(g_kvp_ttrace[kvp_trace_slot()][(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
+#define KVP_TSTAMP(t, e) ((t) < 64 ? (void)(s_kvp_ttrace[(t)][(e)] = ptx::globaltimer_ns()) : (void)0)
 #else
 #define KVP_STAMP(i) ((void)0)
 #define KVP_TSTAMP(t, e) ((void)0)
@@ -108,6 +119,8 @@ struct Params {
     int nrb, nk0, u0, lg_cpb;  // phase 0: row blocks, keys per unit, units per tile, log2(nk0 / 32)
     int p1, n1, rows16;        // phase 1: parts per tile, rows per part, rows rounded up to 16
     int qrows;                 // query rows staged in shared memory (rows rounded up to 64)
+    int nqb;                   // query blocks resident in shared memory (1 or 2)
+    int qreuse;                // every CTA has at most nqb runs: phase 1 reuses phase 0's blocks
     int tiles_per_head, total_tiles, grid, cph, nseg, maxslots;
     int ns, nk, nv;            // ring slots; phase 1 gives K slots [0, nk), V slots [nk, ns)
     float scale2;              // log2(e) / sqrt(d)
@@ -131,7 +144,8 @@ struct SmemBars {
     uint64_t s2full[kS2Ring], s2empty[kS2Ring];     // per S2 ring row: its pieces, its readers
     uint64_t pubfull[2], pubempty[2];               // phase 0 sums of a segment, per buffer
     uint64_t lsefull[2], lseempty[2];               // phase 1 lse2 of a segment, per buffer
-    uint64_t qfull, qempty, fin;
+    uint64_t qfull[2], qempty[2];                   // per query block
+    uint64_t fin;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -147,6 +161,23 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SmemB
                                            const Params& p, int code) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     return ptx::bounded_wait_slow(bar, parity, &sb->abort_flag, p.wait_limit_ns, p.err, code);
+}
+
+// wait_phase with the slow part inline, for the MMA thread: it keeps many values live
+// across its waits, which a call would make it save to local memory.
+__device__ __forceinline__ bool wait_inline(uint64_t* bar, uint32_t parity, SmemBars* sb,
+                                            const Params& p, int code) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (true) {
+        if (ptx::mbar_try_wait_sleep(bar, parity, 20000)) return true;
+        if (*(volatile int*)&sb->abort_flag) return false;
+        if (ptx::globaltimer_ns() - t0 > p.wait_limit_ns) {
+            atomicCAS(p.err, 0, code);
+            *(volatile int*)&sb->abort_flag = 1;
+            return false;
+        }
+    }
 }
 
 // wait_phase for the roles whose warps work as a whole (S2, epilogue): the warp takes one
@@ -165,30 +196,40 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
         if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) return;
 }
 
+// Per 16-bit half: a value whose magnitude is max(|a|, |b|) (its sign is the xor of the
+// inputs' signs, which the caller masks off at the end).
 __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
-    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
-    __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
-    __nv_bfloat162 m = __hmax2(x, y);
-    return *reinterpret_cast<uint32_t*>(&m);
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 // max |v| over the D bf16 values of one row in shared memory, read in 16-byte pieces in a
-// rotated order per lane (consecutive lanes hit distinct bank groups), with four
-// independent running maxima so that the reduction is not one long dependent chain.
+// rotated order per lane (consecutive lanes hit distinct bank groups), eight loads in flight
+// at a time, each piece folded into its own running maximum.
 template <int D>
 __device__ __forceinline__ float row_absmax(const uint8_t* row, int lane) {
     constexpr int kPieces = D * 2 / 16;
+    constexpr int kBatch = 8;
     const uint4* r = reinterpret_cast<const uint4*>(row);
-    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
-#pragma unroll 8
-    for (int c = 0; c < kPieces; ++c) {
-        const uint4 x = r[(c + lane) & (kPieces - 1)];
-        m0 = bf16x2_absmax(m0, x.x & 0x7FFF7FFFu);
-        m1 = bf16x2_absmax(m1, x.y & 0x7FFF7FFFu);
-        m2 = bf16x2_absmax(m2, x.z & 0x7FFF7FFFu);
-        m3 = bf16x2_absmax(m3, x.w & 0x7FFF7FFFu);
+    uint32_t m[kBatch];
+#pragma unroll
+    for (int c = 0; c < kBatch; ++c) m[c] = 0u;
+#pragma unroll
+    for (int c0 = 0; c0 < kPieces; c0 += kBatch) {
+        uint4 x[kBatch];
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) x[c] = r[(c0 + c + lane) & (kPieces - 1)];
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c)
+            m[c] = bf16x2_absmax(m[c], bf16x2_absmax(bf16x2_absmax(x[c].x, x[c].y),
+                                                     bf16x2_absmax(x[c].z, x[c].w)));
     }
-    const uint32_t mx = bf16x2_absmax(bf16x2_absmax(m0, m1), bf16x2_absmax(m2, m3));
+#pragma unroll
+    for (int h = kBatch / 2; h >= 1; h >>= 1)
+#pragma unroll
+        for (int c = 0; c < h; ++c) m[c] = bf16x2_absmax(m[c], m[c + h]);
+    const uint32_t mx = m[0] & 0x7FFF7FFFu;
     return fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
 }
 
@@ -304,7 +345,7 @@ __device__ __forceinline__ float s1_chunk(const float (&v)[32], const float* lse
     return (a0 + a1) + (a2 + a3);
 }
 
-// Phase 1's V stream for a warp of its own (two such warps share it): take the next piece
+// Phase 1's V stream, for warps of their own (two share it): take the next piece
 // (32 keys of a tile) by ticket, wait until its tile has landed and its S2 ring row is
 // free, reduce each key to S2 = max |V| (one key per lane) into the ring, and release the
 // piece's share of the V slot and of the ring row. A worker only ever waits on the barriers
@@ -351,7 +392,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t* Qs = smem;                                  // [D / 64][qrows][64] bf16, 128B swizzle
+    uint8_t* Qs = smem;                                  // [nqb][D / 64][qrows][64] bf16, 128B swizzle
     uint8_t* Slots = smem + p.off_slots;                 // ring slots of tile_bytes each
     float* lse2 = (float*)(smem + p.off_lse);            // [2][rows4]: a segment's lse2 per buffer
     float* comb = (float*)(smem + p.off_comb);           // [kCombBufs][kMaxParts - 1][128]
@@ -369,22 +410,22 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int n = 0;                                      // tiles in this CTA's run
-    int seg_head0 = -1, seg_head1 = -1;             // KV head of each segment's first tile
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
         if (s < p.nseg) {
             uint32_t b, e;
             segment_of_u32(blockIdx.x, s, p.total_tiles, p.grid, p.tiles_per_head, p.cph, b, e);
             n += (int)(e - b);
-            const int h = e > b ? (int)(b / (uint32_t)p.tiles_per_head) : -1;
-            if (s == 0) seg_head0 = h;
-            else seg_head1 = h;
         }
     }
     const int U0 = n * p.u0;                        // phase 0 units of the run
 
     for (int r = threadIdx.x; r < p.rows; r += kThreads) wpos[r] = (uint16_t)(r % p.w);
     if (threadIdx.x == 0) *vclaim = 0u;
+#ifdef KVP_TRACE
+    for (int i = threadIdx.x; i < 64 * 8; i += kThreads) s_kvp_ttrace[i / 8][i % 8] = 0;
+    for (int i = threadIdx.x; i < 64 * 12; i += kThreads) s_kvp_mtrace[i / 12][i % 12] = 0;
+#endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxSlots; ++s) {
             ptx::mbar_init(&sb->kfull[s], 1);
@@ -410,8 +451,10 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             ptx::mbar_init(&sb->lsefull[s], kEpiThreads / 32);
             ptx::mbar_init(&sb->lseempty[s], kEpiThreads / 32);
         }
-        ptx::mbar_init(&sb->qfull, 1);
-        ptx::mbar_init(&sb->qempty, 1);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&sb->qfull[s], 1);
+            ptx::mbar_init(&sb->qempty[s], 1);
+        }
         ptx::mbar_init(&sb->fin, 1);
         sb->abort_flag = 0;
         ptx::fence_mbar_init();
@@ -452,7 +495,9 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         // K is read again by phase 1 (from L2 when it fits); V and phase 1's K stream
         const uint64_t pol_keep = ptx::policy_evict_normal();
         const uint64_t pol_stream = ptx::policy_evict_first();
-        int qgen = 0, cur = -1;
+        // Run r of a phase uses query block r % nqb; when every CTA has at most nqb runs, the
+        // blocks loaded in phase 0 stay for phase 1, else every run loads its block again.
+        int qgen0 = 0, qgen1 = 0;                           // loads into each query block
         // per slot, in registers: bit s = parity of the loads issued to it, and whether any was
         uint32_t kpar = 0, kused = 0, vpar = 0, vused = 0;
         int vs = 0;                                         // next V slot (index s - nk)
@@ -465,17 +510,21 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             CtaRun it(p);
             int head, slot, a, b;
             int i = 0;                                      // tile number within the run
+            int qb = p.nqb - 1;                             // query block of the run
             while (ok && it.next(head, a, b, slot)) {
-                if (head != cur) {
-                    if (qgen > 0 && !(ok = wait_phase(&sb->qempty, (qgen - 1) & 1, sb, p, kErrWaitTma))) break;
-                    ptx::mbar_arrive_expect_tx(&sb->qfull, p.q_bytes);
+                qb ^= p.nqb - 1;
+                if (phase == 0 || !p.qreuse) {
+                    const int qg = qb ? qgen1 : qgen0;
+                    if (qg > 0 && !(ok = wait_phase(&sb->qempty[qb], (qg - 1) & 1, sb, p, kErrWaitTma))) break;
+                    ptx::mbar_arrive_expect_tx(&sb->qfull[qb], p.q_bytes);
                     const int r0 = group_row0(head);
+                    uint8_t* qdst = Qs + (size_t)qb * p.q_bytes;
                     for (int rb = 0; rb < p.qrows; rb += kQBoxRows)
                         for (int c = 0; c < kHalves; ++c)
-                            ptx::tma_load_2d(Qs + c * qhalf + rb * 128, &qmap, &sb->qfull,
+                            ptx::tma_load_2d(qdst + c * qhalf + rb * 128, &qmap, &sb->qfull[qb],
                                              c * 64, r0 + rb, pol_keep);
-                    ++qgen;
-                    cur = head;
+                    if (qb) ++qgen1;
+                    else ++qgen0;
                 }
                 for (int t = a; t < b; ++t, ++i) {
                     const int key0 = (t - head * p.tiles_per_head) * kTile;
@@ -514,14 +563,15 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             if ((kused >> s) & 1) drain_wait(&sb->kfull[s], ((kpar >> s) & 1) ^ 1);
         for (int jv = 0; jv < p.nv; ++jv)
             if ((vused >> jv) & 1) drain_wait(&sb->vfull[jv], ((vpar >> jv) & 1) ^ 1);
-        if (qgen > 0) drain_wait(&sb->qfull, (qgen - 1) & 1);
+        if (qgen0 > 0) drain_wait(&sb->qfull[0], (qgen0 - 1) & 1);
+        if (qgen1 > 0) drain_wait(&sb->qfull[1], (qgen1 - 1) & 1);
       }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t q_addr = ptx::smem_u32(Qs), k_addr = ptx::smem_u32(Slots);
+            const uint32_t q_base = ptx::smem_u32(Qs), k_addr = ptx::smem_u32(Slots);
             const uint32_t idesc0 = ptx::idesc_bf16_f32(128, p.nk0);
-            int qgen = 0, cur = -1;
+            uint32_t qpar = 0;                              // bit b: parity of block b's loads waited for
             uint32_t kpar = 0;                              // bit s: parity of slot s's loads consumed
             uint32_t apar = 0;                              // bit st: parity of stage st's units
             bool ok = true;
@@ -532,23 +582,25 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 int head, slot, a, b;
                 int i = 0;                                  // tile number within the run
                 int unit = 0;                               // unit number within the phase
+                int qb = p.nqb - 1;                         // query block of the run
                 while (ok && it.next(head, a, b, slot)) {
-                    if (head != cur) {
-                        if (!(ok = wait_phase(&sb->qfull, qgen & 1, sb, p, kErrWaitMma))) break;
-                        ++qgen;
-                        cur = head;
+                    qb ^= p.nqb - 1;
+                    if (phase == 0 || !p.qreuse) {
+                        if (!(ok = wait_inline(&sb->qfull[qb], (qpar >> qb) & 1, sb, p, kErrWaitMma))) break;
+                        qpar ^= 1u << qb;
                         ptx::tc_fence_after();
                     }
+                    const uint32_t q_addr = q_base + (uint32_t)qb * p.q_bytes;
                     for (int t = a; t < b && ok; ++t, ++i) {
                         const int s = ks;
                         ks = ks + 1 == kring ? 0 : ks + 1;
-                        if (!(ok = wait_phase(&sb->kfull[s], (kpar >> s) & 1, sb, p, kErrWaitMma))) break;
+                        if (!(ok = wait_inline(&sb->kfull[s], (kpar >> s) & 1, sb, p, kErrWaitMma))) break;
                         KVP_TSTAMP(phase * n + i, 1);
                         const uint32_t kbase = k_addr + s * kSlotBytes;
                         const int nunits = phase == 0 ? p.u0 : p.p1;
                         for (int j = 0; j < nunits; ++j, ++unit) {
                             const int st = unit & (kStages - 1);
-                            if (!(ok = wait_phase(&sb->accempty[st], ((apar >> st) & 1) ^ 1, sb, p, kErrWaitMma))) break;
+                            if (!(ok = wait_inline(&sb->accempty[st], ((apar >> st) & 1) ^ 1, sb, p, kErrWaitMma))) break;
                             apar ^= 1u << st;
                             if (j == 0) KVP_TSTAMP(phase * n + i, 2);
                             ptx::tc_fence_after();
@@ -587,15 +639,8 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         KVP_TSTAMP(phase * n + i, 3);
                     }
                     if (!ok) break;
-                    // release the query rows when the next piece of work (this segment's next
-                    // head, the next segment, or phase 1's first) is another head's
-                    {
-                        int nh;
-                        if (it.t < it.end) nh = it.t / p.tiles_per_head;
-                        else if (it.s + 1 < p.nseg) nh = seg_head1;     // nseg <= 2
-                        else nh = phase == 0 ? seg_head0 : -1;
-                        if (nh >= 0 && nh != cur) ptx::mma_commit(&sb->qempty);
-                    }
+                    // release the query block once its last MMA of this load has completed
+                    if (phase == 1 || !p.qreuse) ptx::mma_commit(&sb->qempty[qb]);
                 }
                 KVP_STAMP(3 + phase);
             }
@@ -771,8 +816,11 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 first_seg = false;
                 const int r0 = group_row0(head);
                 const int nslots = touch * kSlotsPerCta;
-                // four threads per row, each over every fourth slot, in one pass (a running
-                // maximum with the sum rescaled when it rises)
+                // four threads per row, each over every fourth slot, in batches of kMergeBatch
+                // loads issued before any is used (the slots come from L2, whose latency would
+                // otherwise be paid once per slot); per batch, the offset is raised to the
+                // batch's maximum first and the sum rescaled once
+                constexpr int kMergeBatch = 12;
                 for (int rr = (et & 127) >> 2; ; rr += 32) {
                     const int r = ((rr >> 5) * kGroups + eg) * 32 + (rr & 31);
                     if (__all_sync(0xffffffffu, r >= p.rows)) break;
@@ -780,17 +828,22 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                     float M = -INFINITY, S = 0.f;
                     if (r < p.rows) {
                         const float2* pr = p.part + (size_t)(r0 + r) * p.maxslots;
-#pragma unroll 4
-                        for (int sl = q; sl < nslots; sl += 4) {
-                            const float2 ml = __ldcg(pr + sl);
-                            if (ml.y != 0.f) {
-                                if (ml.x > M) {
-                                    S = S * ptx::ex2(M - ml.x) + ml.y;
-                                    M = ml.x;
-                                } else {
-                                    S += ml.y * ptx::ex2(ml.x - M);
-                                }
+                        for (int s0 = q; s0 < nslots; s0 += 4 * kMergeBatch) {
+                            float2 ml[kMergeBatch];
+#pragma unroll
+                            for (int u = 0; u < kMergeBatch; ++u)
+                                ml[u] = s0 + 4 * u < nslots ? __ldcg(pr + s0 + 4 * u) : make_float2(0.f, 0.f);
+                            float Mb = M;
+#pragma unroll
+                            for (int u = 0; u < kMergeBatch; ++u)
+                                if (ml[u].y != 0.f) Mb = fmaxf(Mb, ml[u].x);
+                            if (Mb > M) {
+                                S *= ptx::ex2(M - Mb);             // M = -inf: S is 0 and stays 0
+                                M = Mb;
                             }
+#pragma unroll
+                            for (int u = 0; u < kMergeBatch; ++u)
+                                if (ml[u].y != 0.f) S += ml[u].y * ptx::ex2(ml[u].x - M);
                         }
                     }
 #pragma unroll
@@ -886,6 +939,14 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     if (threadIdx.x == 32 * kWarpEpi) KVP_STAMP(7);
     ptx::tc_fence_before();
     __syncthreads();
+#ifdef KVP_TRACE
+    if (kvp_trace_slot() >= 0) {
+        for (int i = threadIdx.x; i < 64 * 8; i += kThreads)
+            g_kvp_ttrace[kvp_trace_slot()][i / 8][i % 8] = s_kvp_ttrace[i / 8][i % 8];
+        for (int i = threadIdx.x; i < 64 * 12; i += kThreads)
+            g_kvp_mtrace[kvp_trace_slot()][i / 12][i % 12] = s_kvp_mtrace[i / 12][i % 12];
+    }
+#endif
     if (warp == 1) {
         __syncwarp();
         ptx::tc_fence_after();
@@ -957,20 +1018,36 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     // shared memory: Q | ring slots | lse2 [2] | comb | S2 ring | phase 0 hand-off [2] | wpos | barriers
     // (+1 KB to align the base)
     const size_t lse_bytes = 2 * (size_t)((plan.rows + 3) / 4 * 4) * sizeof(float);
-    const size_t comb_bytes = (size_t)kCombBufs * (kMaxParts - 1) * kTile * sizeof(float);
+    const size_t comb_bytes = p.p1 > 1 ? (size_t)kCombBufs * (kMaxParts - 1) * kTile * sizeof(float) : 0;
     const size_t stage_bytes = 2 * (size_t)kGroups * plan.rows * sizeof(float2);
     const size_t s2_bytes = (size_t)kS2Ring * kTile * sizeof(float) + 16;
     const size_t wpos_bytes = (size_t)((plan.rows + 7) / 8 * 8) * sizeof(uint16_t);
     const size_t fixed = lse_bytes + comb_bytes + s2_bytes + stage_bytes + wpos_bytes + kBarBytes + 1024;
-    if (p.q_bytes + fixed > (size_t)kSmemLimit) return false;
-    p.ns = (int)std::min<size_t>(kMaxSlots, ((size_t)kSmemLimit - p.q_bytes - fixed) / p.tile_bytes);
+    // two query blocks (no reload when a CTA changes head) while the ring keeps four slots
+    p.nqb = kMaxQBufs;
+    while (p.nqb > 1 && (size_t)p.nqb * p.q_bytes + fixed + 4 * (size_t)p.tile_bytes > (size_t)kSmemLimit)
+        --p.nqb;
+    const size_t qall = (size_t)p.nqb * p.q_bytes;
+    // whether every CTA's work is at most nqb runs (a run: consecutive tiles of one head)
+    p.qreuse = 1;
+    for (int c = 0; c < p.grid && p.qreuse; ++c) {
+        int runs = 0;
+        for (int sg = 0; sg < p.nseg; ++sg) {
+            long long b, e;
+            segment_of(c, sg, p.total_tiles, p.grid, p.tiles_per_head, p.cph, b, e);
+            if (e > b) runs += (int)((e - 1) / p.tiles_per_head - b / p.tiles_per_head + 1);
+        }
+        if (runs > p.nqb) p.qreuse = 0;
+    }
+    if (qall + fixed > (size_t)kSmemLimit) return false;
+    p.ns = (int)std::min<size_t>(kMaxSlots, ((size_t)kSmemLimit - qall - fixed) / p.tile_bytes);
     if (p.ns < 2) return false;
     // phase 0 streams K through every slot; phase 1 gives V (from HBM) the deeper share and
     // K (mostly from L2) two slots, or one when the ring is short
     p.nk = p.ns >= 4 ? 2 : 1;
     p.nv = p.ns - p.nk;
     if (p.nv < 1) return false;
-    p.off_slots = p.q_bytes;
+    p.off_slots = (uint32_t)qall;
     uint32_t off = p.off_slots + (uint32_t)p.ns * p.tile_bytes;
     p.off_lse = off;
     off += (uint32_t)lse_bytes;
