@@ -256,8 +256,8 @@ def workload_config(wl, l2_note):
 
 
 def measure_extra_paths(kvp, torch, sh, wl, sets, bufs, dev, stream, peak, n=40):
-    """Per-call device times (CUDA events on the launching stream, median of n calls after
-    warm-up, outside the timed region) of the calls beside the headline path, on the same
+    """Per-call device times (CUDA events on the launching stream around a replayed graph
+    of back-to-back calls, outside the timed region) of the calls beside the headline path, on the same
     workload: the policy selection (sinks, S1 pooling), the CurDKV leverage scorer (r = 20,
     rotating input sets larger than L2), the adaptive per-head budgets (alpha = 0.20) and
     the ragged compaction."""
@@ -277,27 +277,47 @@ def measure_extra_paths(kvp, torch, sh, wl, sets, bufs, dev, stream, peak, n=40)
     v_out = torch.empty_like(k_out)
     pol = kvp.make_policy(4, 7, kvp.RANK_PRODUCT)
 
-    def timed(fn):
+    def timed(fn, reps=8, replays=10):
+        # device time per call: a CUDA graph of `reps` back-to-back calls, replayed between
+        # two events on the launching stream (host-launched calls, median, if capture fails)
         for i in range(3):
             fn(i)
         torch.cuda.synchronize(dev)
-        ts = []
-        for i in range(n):
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
+                for i in range(reps):
+                    fn(i)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize(dev)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            fn(i)
+            for _ in range(replays):
+                g.replay()
             e1.record(stream)
             torch.cuda.synchronize(dev)
-            ts.append(e0.elapsed_time(e1))
-        return float(np.median(ts))
+            del g
+            return e0.elapsed_time(e1) / (reps * replays)
+        except Exception:
+            ts = []
+            for i in range(n):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn(i)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1))
+            return float(np.median(ts))
 
+    cur = lambda: torch.cuda.current_stream(dev)      # the capturing stream inside a graph
     nsets = len(sets)
-    t_pol = timed(lambda i: kvp.kvp_select_policy(sh, pol, s1, s2, idx, stream))
+    t_pol = timed(lambda i: kvp.kvp_select_policy(sh, pol, s1, s2, idx, cur()))
     t_lev = timed(lambda i: kvp.kvp_leverage(sh, sets[i % nsets][1], sets[i % nsets][2], g, lev,
-                                             bufs[i % nsets].workspace, stream))
-    t_ada = timed(lambda i: kvp.kvp_select_adaptive(sh, 0.2, buf.score, aidx, counts, aws, stream))
+                                             bufs[i % nsets].workspace, cur()))
+    t_ada = timed(lambda i: kvp.kvp_select_adaptive(sh, 0.2, buf.score, aidx, counts, aws, cur()))
     t_rag = timed(lambda i: kvp.kvp_compact_ragged(sh, sets[i % nsets][1], sets[i % nsets][2], aidx,
-                                                   counts, k_out, v_out, stream))
+                                                   counts, k_out, v_out, cur()))
     lev_bytes = 2 * b * hkv * L * d * 2 + b * hkv * L * 4 * 3          # K, V; score written, scaled
     rag_bytes = 2 * 2 * b * hkv * B * d * 2 + b * hkv * B * 4          # rows read + written; idx
     return {

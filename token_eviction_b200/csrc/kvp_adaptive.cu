@@ -118,6 +118,8 @@ gather_ragged(const uint4* __restrict__ k, const uint4* __restrict__ v, const in
               const int32_t* __restrict__ counts, uint4* __restrict__ k_out, uint4* __restrict__ v_out,
               int hkv, int L, int B, int pieces) {
     extern __shared__ int32_t offs[];                     // [hkv + 1] row offsets of the heads
+    constexpr int kPer = 4;                               // 16-byte pieces of K (and of V) per item
+    asm volatile("griddepcontrol.wait;" ::: "memory");    // the indices' producer has completed
     const int b = blockIdx.y;
     if (threadIdx.x == 0) {
         int o = 0;
@@ -128,29 +130,35 @@ gather_ragged(const uint4* __restrict__ k, const uint4* __restrict__ v, const in
         offs[hkv] = o;
     }
     __syncthreads();
-    const long long rows = offs[hkv];                     // hkv B when the counts are consistent
-    const long long items = rows * pieces;
+    const long long rows = min((long long)offs[hkv], (long long)hkv * B);   // hkv B when consistent
+    const int ipr = pieces / kPer;                        // items per row
+    const long long items = rows * ipr;
     for (long long i = blockIdx.x * 256ll + threadIdx.x; i < items; i += (long long)gridDim.x * 256) {
-        const long long r = i / pieces;
-        const int c = (int)(i - r * pieces);
-        if (r >= (long long)hkv * B) break;
+        const long long r = i / ipr;
+        const int c = (int)(i - r * ipr) * kPer;
         int lo = 0, hi = hkv - 1;                         // the head whose rows hold r
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (offs[mid] <= r) lo = mid;
             else hi = mid - 1;
         }
-        const int j = idx[(size_t)b * hkv * B + r];
+        const int j = __ldg(idx + (size_t)b * hkv * B + r);
         const size_t dst = ((size_t)b * hkv * B + r) * pieces + c;
+        uint4 ka[kPer], va[kPer];
         if (j >= 0 && j < L) {
             const size_t src = (((size_t)b * hkv + lo) * L + j) * pieces + c;
-            const uint4 kv = __ldg(k + src), vv = __ldg(v + src);
-            k_out[dst] = kv;
-            v_out[dst] = vv;
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) ka[q] = __ldg(k + src + q);
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) va[q] = __ldg(v + src + q);
         } else {
-            k_out[dst] = make_uint4(0, 0, 0, 0);
-            v_out[dst] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) ka[q] = va[q] = make_uint4(0, 0, 0, 0);
         }
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) __stcs(k_out + dst + q, ka[q]);
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) __stcs(v_out + dst + q, va[q]);
     }
 }
 
@@ -207,12 +215,22 @@ cudaError_t launch_compact_ragged(const kvp_shape& s, const uint16_t* k, const u
     const int pieces = s.head_dim * 2 / 16;
     const long long items = (long long)s.hkv * s.budget * pieces;
     const int sms = std::max(1, num_sms());
-    const int gx = (int)std::max<long long>(1, std::min<long long>((items + 255) / 256,
-                                                                   std::max(1, sms * 8 / s.batch)));
-    gather_ragged<<<dim3(gx, s.batch), 256, (s.hkv + 1) * sizeof(int32_t), st>>>(
-        (const uint4*)k, (const uint4*)v, idx, counts, (uint4*)k_out, (uint4*)v_out, s.hkv, s.seq_len,
-        s.budget, pieces);
-    return cudaPeekAtLastError();
+    // four 16-byte pieces per thread and per row: whole waves over the SMs, at most 8 CTAs each
+    const long long want = (items / 4 + 255) / 256;
+    const long long per_b = std::max(1, sms * 8 / s.batch);
+    const int gx = (int)std::max<long long>(1, std::min<long long>(want, per_b));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)gx, (unsigned)s.batch);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = (s.hkv + 1) * sizeof(int32_t);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlaps the launch
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gather_ragged, (const uint4*)k, (const uint4*)v, idx, counts,
+                              (uint4*)k_out, (uint4*)v_out, s.hkv, s.seq_len, s.budget, pieces);
 }
 
 #ifdef KVP_CHECKS
