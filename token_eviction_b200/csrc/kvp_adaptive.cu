@@ -131,34 +131,45 @@ gather_ragged(const uint4* __restrict__ k, const uint4* __restrict__ v, const in
     }
     __syncthreads();
     const long long rows = min((long long)offs[hkv], (long long)hkv * B);   // hkv B when consistent
-    const int ipr = pieces / kPer;                        // items per row
-    const long long items = rows * ipr;
-    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < items; i += (long long)gridDim.x * 256) {
-        const long long r = i / ipr;
-        const int c = (int)(i - r * ipr) * kPer;
-        int lo = 0, hi = hkv - 1;                         // the head whose rows hold r
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (offs[mid] <= r) lo = mid;
-            else hi = mid - 1;
+    const long long total = rows * pieces;                // output pieces of this sequence
+    const int lane = threadIdx.x & 31;
+    const int ps = __ffs(pieces) - 1;                     // pieces per row: a power of two
+    const long long nwarps = (long long)gridDim.x * 8;
+    // each warp a block of 32 kPer consecutive pieces; lane l takes l, l + 32, l + 64, l + 96
+    for (long long w = blockIdx.x * 8ll + (threadIdx.x >> 5); w * 32 * kPer < total; w += nwarps) {
+        long long e[kPer];
+        int j[kPer], h[kPer];
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            e[q] = w * 32 * kPer + q * 32 + lane;
+            const long long r = e[q] >> ps;
+            int lo = 0, hi = hkv - 1;                     // the head whose rows hold r
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (offs[mid] <= r) lo = mid;
+                else hi = mid - 1;
+            }
+            h[q] = lo;
+            j[q] = e[q] < total ? __ldg(idx + (size_t)b * hkv * B + r) : -1;
         }
-        const int j = __ldg(idx + (size_t)b * hkv * B + r);
-        const size_t dst = ((size_t)b * hkv * B + r) * pieces + c;
         uint4 ka[kPer], va[kPer];
-        if (j >= 0 && j < L) {
-            const size_t src = (((size_t)b * hkv + lo) * L + j) * pieces + c;
 #pragma unroll
-            for (int q = 0; q < kPer; ++q) ka[q] = __ldg(k + src + q);
-#pragma unroll
-            for (int q = 0; q < kPer; ++q) va[q] = __ldg(v + src + q);
-        } else {
-#pragma unroll
-            for (int q = 0; q < kPer; ++q) ka[q] = va[q] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < kPer; ++q) {
+            if (e[q] < total && j[q] >= 0 && j[q] < L) {
+                const size_t src = ((((size_t)b * hkv + h[q]) * L + j[q]) << ps) + (e[q] & (pieces - 1));
+                ka[q] = __ldg(k + src);
+                va[q] = __ldg(v + src);
+            } else {
+                ka[q] = va[q] = make_uint4(0, 0, 0, 0);
+            }
         }
 #pragma unroll
-        for (int q = 0; q < kPer; ++q) __stcs(k_out + dst + q, ka[q]);
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) __stcs(v_out + dst + q, va[q]);
+        for (int q = 0; q < kPer; ++q) {
+            if (e[q] >= total) continue;
+            const size_t dst = (size_t)b * hkv * B * pieces + e[q];
+            __stcs(k_out + dst, ka[q]);
+            __stcs(v_out + dst, va[q]);
+        }
     }
 }
 
