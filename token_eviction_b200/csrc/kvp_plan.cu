@@ -57,9 +57,16 @@ bool plan_of(const kvp_shape& s, Plan* p) {
             p->grid = (int)(cph * units);
         }
     }
+    // Two segments change head twice more per CTA. The scoring kernel keeps both runs'
+    // query blocks in shared memory when they fit beside four 128-key ring slots (and some
+    // 24 KiB of bookkeeping); otherwise every change of head reloads a block, which costs
+    // about as much as kHeadSwitchTiles tiles (GQA-7 with w = 64: 112 KiB per block).
+    const long long qblock = (long long)(p->rows + 63) / 64 * 64 * s.head_dim * 2;
+    const long long tile = 128LL * s.head_dim * 2;
+    const bool both_blocks = 2 * qblock + 4 * tile + 24 * 1024 <= 227 * 1024;
     if (units % 2 == 0 && units <= 2 * kPlanGrid) {
         const long long cph = std::min<long long>(2 * kPlanGrid / units, tph);
-        const long long cost = 2 * ((tph + cph - 1) / cph);
+        const long long cost = 2 * ((tph + cph - 1) / cph) + (both_blocks ? 0 : kHeadSwitchTiles);
         if (cost <= best_cost) {
             best_cost = cost;
             p->cph = (int)cph;

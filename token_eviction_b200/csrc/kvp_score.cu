@@ -116,7 +116,7 @@ enum : int { kErrWaitTma = 1, kErrWaitMma = 2, kErrWaitEpi = 3, kErrWaitPeers = 
 
 struct Params {
     int L, w, rows, hq, hkv, G;
-    int nrb, nk0, u0, lg_cpb;  // phase 0: row blocks, keys per unit, units per tile, log2(nk0 / 32)
+    int nrb, u0;               // phase 0: row blocks of 128 query rows; units per tile (one per block)
     int p1, n1, rows16;        // phase 1: parts per tile, rows per part, rows rounded up to 16
     int qrows;                 // query rows staged in shared memory (rows rounded up to 64)
     int nqb;                   // query blocks resident in shared memory (1 or 2)
@@ -570,7 +570,7 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t q_base = ptx::smem_u32(Qs), k_addr = ptx::smem_u32(Slots);
-            const uint32_t idesc0 = ptx::idesc_bf16_f32(128, p.nk0);
+            const uint32_t idesc0 = ptx::idesc_bf16_f32(128, kTile);
             uint32_t qpar = 0;                              // bit b: parity of block b's loads waited for
             uint32_t kpar = 0;                              // bit s: parity of slot s's loads consumed
             uint32_t apar = 0;                              // bit st: parity of stage st's units
@@ -606,17 +606,15 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                             ptx::tc_fence_after();
                             const uint32_t d0 = tmem + (uint32_t)(st * kStageCols);
                             if (phase == 0) {
-                                // D[row, key] for every row block: A = Q rows, B = the unit's keys
-#pragma unroll 1
-                                for (int rb = 0; rb < p.nrb; ++rb) {
-                                    const uint64_t qd = ptx::sw128_kmajor_desc(q_addr + rb * 128 * 128);
-                                    const uint64_t kd = ptx::sw128_kmajor_desc(kbase + j * p.nk0 * 128);
+                                // D[row, key] for row block j and the tile's 128 keys: A = Q rows,
+                                // B = the K tile (each operand read once per unit)
+                                const uint64_t qd = ptx::sw128_kmajor_desc(q_addr + j * 128 * 128);
+                                const uint64_t kd = ptx::sw128_kmajor_desc(kbase);
 #pragma unroll
-                                    for (int ks = 0; ks < D / 16; ++ks) {
-                                        const uint32_t qo = ((ks >> 2) * qhalf + (ks & 3) * 32) >> 4;
-                                        const uint32_t ko = ((ks >> 2) * kHalfTile + (ks & 3) * 32) >> 4;
-                                        ptx::mma_bf16_ss(d0 + rb * p.nk0, qd + qo, kd + ko, idesc0, ks > 0);
-                                    }
+                                for (int ks = 0; ks < D / 16; ++ks) {
+                                    const uint32_t qo = ((ks >> 2) * qhalf + (ks & 3) * 32) >> 4;
+                                    const uint32_t ko = ((ks >> 2) * kHalfTile + (ks & 3) * 32) >> 4;
+                                    ptx::mma_bf16_ss(d0, qd + qo, kd + ko, idesc0, ks > 0);
                                 }
                             } else {
                                 // D[key, row] for one part of the query rows: A = keys, B = Q rows
@@ -704,11 +702,6 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         // ---- phase 0: per query row, the running offset and sum of 2^(t - m) over the keys
         //      of this group's units (thread = row, TMEM columns = keys)
         {
-            // chunks of a unit that hold rows of this warp: all rows of a row block are live
-            // or none, and live chunks are a prefix of the unit's four
-            const int rbl = p.rows > quarter * 32 ? min(p.nrb, (p.rows - quarter * 32 + 127) / 128) : 0;
-            const int nl = min(4, rbl << p.lg_cpb);
-            const int cmask = (1 << p.lg_cpb) - 1;
             CtaRun it(p);
             int head, slot, a, b;
             int unit = 0, i = 0, k = 0;
@@ -722,17 +715,18 @@ score_fused_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                         if (!(ok = wait_warp(&sb->accfull[eg], (unit / kStages) & 1, sb, p, kErrWaitEpi))) break;
                         if (lq == 0) KVP_TSTAMP(i, 4);
                         ptx::tc_fence_after();
-                        const int kbase = key_t + j * p.nk0;
-                        // chunk c: TMEM columns [32c, 32c + 32) of the stage, row block c >> lg_cpb,
-                        // keys kbase + 32 (c & cmask) + e
+                        // unit j is row block j; chunk c: TMEM columns [32c, 32c + 32) of the
+                        // stage, keys key_t + 32 c + e. A warp whose rows of the block all lie
+                        // beyond the group's rows skips it (rows past the last are not published)
+                        const int rb = j;
+                        const int nl = rb * 128 + quarter * 32 < p.rows ? 4 : 0;
 #pragma unroll 1
                         for (int c = 0; c < nl; ++c) {
                             float v[32];
                             __syncwarp();
                             ptx::tmem_ld_32x32b_x32(tst + c * 32, v);
                             ptx::tmem_ld_wait(v);
-                            const int rb = c >> p.lg_cpb;
-                            const int j0 = kbase + ((c & cmask) << 5);
+                            const int j0 = key_t + (c << 5);
                             if (j0 + 31 > window0) {         // window or ragged keys: mask per row
                                 // the row's last visible key is window0 + its window position
                                 const int rel = window0 + (rb * 128 + lq) % p.w - j0;
@@ -981,12 +975,10 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.rows = plan.rows;
     p.hq = s.hq;
     p.hkv = s.hkv;
-    // phase 0: row blocks of 128 query rows; a unit covers nk0 keys of every row block in
-    // 128 TMEM columns (4 chunks of 32 per thread)
+    // phase 0: row blocks of 128 query rows; unit j of a tile covers row block j and the
+    // tile's 128 keys in 128 TMEM columns (4 chunks of 32 per thread)
     p.nrb = (plan.rows + 127) / 128;
-    p.nk0 = p.nrb == 1 ? 128 : p.nrb == 2 ? 64 : 32;
-    p.u0 = kTile / p.nk0;
-    p.lg_cpb = p.nk0 == 128 ? 2 : p.nk0 == 64 ? 1 : 0;
+    p.u0 = p.nrb;
     // phase 1: the query rows in p1 parts of n1 (a multiple of 16, at most 128) rows
     p.rows16 = (plan.rows + 15) / 16 * 16;
     p.p1 = (p.rows16 + kStageCols - 1) / kStageCols;
@@ -1027,18 +1019,22 @@ bool build_launch(const kvp_shape& s, const Plan& plan, int sms, Launch* L) {
     p.nqb = kMaxQBufs;
     while (p.nqb > 1 && (size_t)p.nqb * p.q_bytes + fixed + 4 * (size_t)p.tile_bytes > (size_t)kSmemLimit)
         --p.nqb;
-    const size_t qall = (size_t)p.nqb * p.q_bytes;
-    // whether every CTA's work is at most nqb runs (a run: consecutive tiles of one head)
-    p.qreuse = 1;
-    for (int c = 0; c < p.grid && p.qreuse; ++c) {
+    // the most runs any CTA has (a run: consecutive tiles of one head); one block is enough
+    // when no CTA changes head
+    int max_runs = 0;
+    for (int c = 0; c < p.grid; ++c) {
         int runs = 0;
         for (int sg = 0; sg < p.nseg; ++sg) {
             long long b, e;
             segment_of(c, sg, p.total_tiles, p.grid, p.tiles_per_head, p.cph, b, e);
             if (e > b) runs += (int)((e - 1) / p.tiles_per_head - b / p.tiles_per_head + 1);
         }
-        if (runs > p.nqb) p.qreuse = 0;
+        max_runs = std::max(max_runs, runs);
     }
+    if (max_runs <= 1) p.nqb = 1;
+    const size_t qall = (size_t)p.nqb * p.q_bytes;
+    // phase 1 reuses phase 0's blocks when every CTA has at most nqb runs
+    p.qreuse = max_runs <= p.nqb ? 1 : 0;
     if (qall + fixed > (size_t)kSmemLimit) return false;
     p.ns = (int)std::min<size_t>(kMaxSlots, ((size_t)kSmemLimit - qall - fixed) / p.tile_bytes);
     if (p.ns < 2) return false;
