@@ -122,3 +122,10 @@ def test_run_cuts_and_owner_lookup_agree(tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, out.stdout + out.stderr
     assert "0 bad" in out.stdout
+    plans = dict(line.split(": ", 1) for line in out.stdout.splitlines() if line.startswith("plan "))
+    # the 32K layer: two head-aligned segments per CTA (both 32 KiB query blocks stay in
+    # shared memory), 37 parts per head on 148 CTAs
+    assert plans["plan b1 hkv8 L32768"] == "grid 148 cph 37 nseg 2"
+    # GQA-7 (G w = 448: 112 KiB query blocks, too big to keep two): one segment per CTA,
+    # so that no CTA changes head and reloads its block
+    assert plans["plan b8 hkv4 L16384"].endswith("nseg 1")
